@@ -1,0 +1,329 @@
+"""CPU oracle for CubicQuant weight-only GEMM -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding in ``bit_non_uniform_b200``) never does.
+
+The arithmetic lives in ``cq_oracle.c`` (plain C, FP64, naive loops); this
+module only marshals numpy arrays into it, and orchestrates the MoE layer as
+the plain composition of those calls.  Source of the method: the ModelScope
+article "CubicQuant：用三次曲线重塑低比特量化，Kimi K3 2.5Bit 模型首发实践"
+(sections "CubicQuant 核心" for the format, "存储开销是透明的：B+64/G bit" for
+the storage identity, "从曲线到量化器：数据无关的组内拟合" for the fitter and
+"压缩权重必须“边解码、边计算”" for the A16 execution path).
+
+Parity status: every function here is pinned by a not-gpu test in
+``tests/test_oracle_*.py`` except the fitter's *midrise* statistics, which
+the article does not pin (its W4 G128 table is reproduced in midtread mode).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+MIDRISE = 0
+MIDTREAD = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "cq_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile cq_oracle.c into liboracle.so (gcc, no FMA contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    ):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-ffp-contract=off", "-fPIC", "-shared", "-pthread",
+             _SRC, "-o", tmp, "-lm"]
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB_PATH)
+    P = ctypes.c_void_p
+    i64, i32, dbl, flt = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_float
+    u16 = ctypes.c_uint16
+    sig = {
+        "cqo_half_to_double": (dbl, [u16]),
+        "cqo_double_to_half": (u16, [dbl]),
+        "cqo_float_to_bf16": (u16, [flt]),
+        "cqo_bf16_to_double": (dbl, [u16]),
+        "cqo_pack": (None, [P, i64, i64, i32, P]),
+        "cqo_unpack": (None, [P, i64, i64, i32, P]),
+        "cqo_q": (dbl, [dbl, dbl, dbl]),
+        "cqo_level": (dbl, [i32, i32, i32, flt, u16, u16]),
+        "cqo_levels": (None, [i32, i32, flt, u16, u16, P]),
+        "cqo_is_monotone": (i32, [u16, u16]),
+        "cqo_decode": (None, [P, P, P, i64, i64, i32, i32, i32, P, P, P]),
+        "cqo_gemm": (None, [P, i64, P, P, P, i64, i64, i32, i32, i32, P, P, i32]),
+        "cqo_nearest": (i32, [P, i32, dbl]),
+        "cqo_nearest_bruteforce": (i32, [P, i32, dbl]),
+        "cqo_fit": (None, [P, i64, i32, i32, i32, P, i32, P, i32, P, i32, i32,
+                           P, P, P, P, P, i32]),
+        "cqo_optimal_sse": (dbl, [P, i32, i32]),
+        "cqo_num_threads": (i32, [i32]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# --------------------------------------------------------------------------
+# number helpers
+# --------------------------------------------------------------------------
+
+def half_to_double(h: int) -> float:
+    return _load().cqo_half_to_double(int(h))
+
+
+def double_to_half(x: float) -> int:
+    return int(_load().cqo_double_to_half(float(x)))
+
+
+def float_to_bf16(x: float) -> int:
+    return int(_load().cqo_float_to_bf16(float(x)))
+
+
+def bf16_to_double(h: int) -> float:
+    return _load().cqo_bf16_to_double(int(h))
+
+
+def num_threads() -> int:
+    return int(_load().cqo_num_threads(0))
+
+
+# --------------------------------------------------------------------------
+# format
+# --------------------------------------------------------------------------
+
+def bits_per_weight(B: int, G: int) -> float:
+    """Storage per weight: G*B payload bits + 32 (FP32 s) + 32 (two FP16) per
+    group, i.e. B + 64/G bits ("存储开销是透明的：B+64/G bit")."""
+    return (G * B + 32 + 32) / G
+
+
+def pack(codes: np.ndarray, B: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    N, K = codes.shape
+    assert (K * B) % 8 == 0
+    out = np.empty((N, K * B // 8), dtype=np.uint8)
+    _load().cqo_pack(_ptr(codes), N, K, B, _ptr(out))
+    return out
+
+
+def unpack(packed: np.ndarray, K: int, B: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    N = packed.shape[0]
+    out = np.empty((N, K), dtype=np.uint8)
+    _load().cqo_unpack(_ptr(packed), N, K, B, _ptr(out))
+    return out
+
+
+def q(t: float, a: float, b: float) -> float:
+    return _load().cqo_q(float(t), float(a), float(b))
+
+
+def level(u: int, B: int, mode: int, s: float, a_h: int, b_h: int) -> float:
+    return _load().cqo_level(int(u), B, mode, float(s), int(a_h), int(b_h))
+
+
+def levels(B: int, mode: int, s: float, a_h: int, b_h: int) -> np.ndarray:
+    out = np.empty(1 << B, dtype=np.float64)
+    _load().cqo_levels(B, mode, float(s), int(a_h), int(b_h), _ptr(out))
+    return out
+
+
+def is_monotone(a_h: int, b_h: int) -> bool:
+    return bool(_load().cqo_is_monotone(int(a_h), int(b_h)))
+
+
+def decode(packed, scales, ab, N, K, B, G, mode=MIDRISE):
+    """Returns (w64, w32, w16bits): exact FP64 levels, FP32 and BF16 roundings."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    ab = np.ascontiguousarray(ab, dtype=np.uint16)
+    w64 = np.empty((N, K), dtype=np.float64)
+    w32 = np.empty((N, K), dtype=np.float32)
+    w16 = np.empty((N, K), dtype=np.uint16)
+    _load().cqo_decode(_ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G, mode,
+                       _ptr(w64), _ptr(w32), _ptr(w16))
+    return w64, w32, w16
+
+
+def gemm(x_bf16bits, packed, scales, ab, N, K, B, G, mode=MIDRISE, nthreads=0):
+    """y[m][n] = sum_k x[m][k] w[n][k] in FP64 and bound = sum_k |x w|.
+
+    x_bf16bits: uint16 [M][K] (bfloat16 bit patterns)."""
+    x = np.ascontiguousarray(x_bf16bits, dtype=np.uint16)
+    M = x.shape[0]
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    ab = np.ascontiguousarray(ab, dtype=np.uint16)
+    y = np.empty((M, N), dtype=np.float64)
+    bound = np.empty((M, N), dtype=np.float64)
+    _load().cqo_gemm(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G,
+                     mode, _ptr(y), _ptr(bound), nthreads)
+    return y, bound
+
+
+def silu(g):
+    """silu(g) = g / (1 + exp(-g)), FP64."""
+    g = np.asarray(g, dtype=np.float64)
+    return g / (1.0 + np.exp(-g))
+
+
+def swiglu(y: np.ndarray) -> np.ndarray:
+    """SwiGLU over the two halves of the last axis: gate = first half,
+    up = second half, h = silu(gate) * up (FP64)."""
+    n2 = y.shape[-1] // 2
+    return silu(y[..., :n2]) * y[..., n2:]
+
+
+def bf16_round(v: np.ndarray) -> np.ndarray:
+    """FP64 -> FP32 (RNE) -> BF16 (RNE); returns the uint16 bit patterns."""
+    f = np.ascontiguousarray(np.asarray(v, dtype=np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    nan = (u & 0x7F800000) == 0x7F800000
+    nan &= (u & 0x007FFFFF) != 0
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+    r[nan] = 0x7FC0
+    return r
+
+
+def bf16_bits_to_f64(h: np.ndarray) -> np.ndarray:
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    return (h.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# MoE layer: the composition gate/up -> SwiGLU -> down -> weighted combine
+# --------------------------------------------------------------------------
+
+def moe_routes(tokens_bf16bits, topk_ids, experts, H, I, G, mode=MIDRISE,
+               routes=None, nthreads=0):
+    """Per-route outputs of the routed-expert FFN, FP64.
+
+    experts[e] = dict(B_gu, packed_gu [2I][H*B/8], scales_gu, ab_gu,
+                      B_dn, packed_dn [H][I*B/8], scales_dn, ab_dn)
+    (a callable e -> dict is accepted too, so large layers can be
+    regenerated one expert at a time).
+    Route r = (t, j) uses expert topk_ids[t][j]:
+        gu = W_gu x_t (2I outputs), h = bf16(silu(gu[:I]) * gu[I:]),
+        y_r = W_dn h (H outputs).
+    h is rounded to BF16 because the GPU chain stores it in BF16.
+    routes: optional list of flat route indices r = t*k + j to evaluate.
+    Returns dict r -> (y_r [H] float64, bound_r [H] float64)."""
+    T, k = topk_ids.shape
+    if routes is None:
+        routes = range(T * k)
+    by_expert: dict[int, list[int]] = {}
+    for r in routes:
+        e = int(topk_ids[r // k, r % k])
+        by_expert.setdefault(e, []).append(int(r))
+    get = experts if callable(experts) else (lambda e: experts[e])
+    out = {}
+    for e in sorted(by_expert):
+        rs = by_expert[e]
+        ex = get(e)
+        xs = np.ascontiguousarray(tokens_bf16bits[[r // k for r in rs]])
+        gu, _ = gemm(xs, ex["packed_gu"], ex["scales_gu"], ex["ab_gu"], 2 * I, H,
+                     ex["B_gu"], G, mode, nthreads)
+        h = bf16_round(swiglu(gu))
+        y, bnd = gemm(h, ex["packed_dn"], ex["scales_dn"], ex["ab_dn"], H, I,
+                      ex["B_dn"], G, mode, nthreads)
+        for i, r in enumerate(rs):
+            out[r] = (y[i], bnd[i])
+    return out
+
+
+def moe_combine(route_out, topk_w, tokens=None):
+    """out[t] = sum_j w[t][j] * y_(t,j) in FP64 (j ascending); also returns
+    the matching bound sum_j |w| * bound_(t,j)."""
+    T, k = topk_w.shape
+    tokens = range(T) if tokens is None else tokens
+    res = {}
+    for t in tokens:
+        acc = None
+        bnd = None
+        for j in range(k):
+            y, b = route_out[t * k + j]
+            w = float(topk_w[t, j])
+            acc = w * y if acc is None else acc + w * y
+            bnd = abs(w) * b if bnd is None else bnd + abs(w) * b
+        res[t] = (acc, bnd)
+    return res
+
+
+# --------------------------------------------------------------------------
+# fitter
+# --------------------------------------------------------------------------
+
+def default_grids():
+    """Candidate grids of the data-free fitter (the article gives none):
+    a in [1/16, 5/2] and b in [-2, 2], both in steps of 1/16 (all exact in
+    FP16), clip ratio alpha in {0.30, 0.31, ..., 1.00}."""
+    a = np.arange(1, 41, dtype=np.float64) / 16.0
+    b = np.arange(-32, 33, dtype=np.float64) / 16.0
+    alpha = np.round(np.arange(30, 101, dtype=np.float64)) / 100.0
+    return a, b, alpha
+
+
+def fit(w: np.ndarray, G: int, B: int, mode=MIDRISE, uniform_only=False,
+        grids=None, nthreads=0):
+    """Fit every group of w (flattened, length multiple of G).
+
+    Returns dict(codes [ng][G] uint8, s [ng] f32, ab [ng][2] fp16 bits,
+    sse [ng], clipped [ng])."""
+    w = np.ascontiguousarray(np.asarray(w, dtype=np.float64).reshape(-1, G))
+    ng = w.shape[0]
+    a, b, alpha = grids if grids is not None else default_grids()
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    b = np.ascontiguousarray(b, dtype=np.float64)
+    alpha = np.ascontiguousarray(alpha, dtype=np.float64)
+    codes = np.empty((ng, G), dtype=np.uint8)
+    s = np.empty(ng, dtype=np.float32)
+    ab = np.empty((ng, 2), dtype=np.uint16)
+    sse = np.empty(ng, dtype=np.float64)
+    clipped = np.empty(ng, dtype=np.int32)
+    _load().cqo_fit(_ptr(w), ng, G, B, mode, _ptr(a), len(a), _ptr(b), len(b),
+                    _ptr(alpha), len(alpha), int(uniform_only), _ptr(codes), _ptr(s),
+                    _ptr(ab), _ptr(sse), _ptr(clipped), nthreads)
+    return dict(codes=codes, s=s, ab=ab, sse=sse, clipped=clipped)
+
+
+def nrmse(sse: np.ndarray, w: np.ndarray) -> float:
+    """Group reconstruction error normalised by source weight energy,
+    sqrt(sum SSE / sum w^2) over the tensor."""
+    return float(np.sqrt(np.sum(sse) / np.sum(np.asarray(w, dtype=np.float64) ** 2)))
+
+
+def nearest(levels_sorted: np.ndarray, v: float, brute: bool = False) -> int:
+    lv = np.ascontiguousarray(levels_sorted, dtype=np.float64)
+    f = _load().cqo_nearest_bruteforce if brute else _load().cqo_nearest
+    return int(f(_ptr(lv), len(lv), float(v)))
+
+
+def optimal_sse(v: np.ndarray, nlev: int) -> float:
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    return float(_load().cqo_optimal_sse(_ptr(v), len(v), nlev))

@@ -1,0 +1,544 @@
+/*
+ * cq_oracle.c -- CPU reference ("oracle") for CubicQuant weight-only GEMM.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may link, load or
+ * call this file: only the test-suite, the smoke check and the benchmark's
+ * CPU-baseline leg use it.  It is deliberately plain and slow: FP64
+ * arithmetic, naive loops, no blocking, no reordering of any sum beyond the
+ * definitions below.  It shares no code with the CUDA library.
+ *
+ * Source of the method: the ModelScope article "CubicQuant：用三次曲线重塑低
+ * 比特量化，Kimi K3 2.5Bit 模型首发实践" (cited below as [CQ]), sections
+ *   [CQ core]    "CubicQuant 核心：把直线网格“掰弯”"   (format and decode)
+ *   [CQ two]     "为什么只用两个形状参数？"              (dense code stream)
+ *   [CQ bits]    "存储开销是透明的：B+64/G bit"          (storage identity)
+ *   [CQ fit]     "从曲线到量化器：数据无关的组内拟合"     (group fitter)
+ *   [CQ fused]   "压缩权重必须“边解码、边计算”"          (A16 execution)
+ *
+ * The article's displayed formulas were lost when the page was extracted;
+ * the readings used here are:
+ *   - code u in [0, 2^B-1], MIDRISE grid (the build contract):
+ *       Kc = (2^B-1)/2, k = u - Kc, t = |k|/Kc, sign(k) never 0;
+ *   - MIDTREAD grid (sign-magnitude alternative, also supported):
+ *       Kc = 2^(B-1)-1, k = u - Kc, t = |k|/Kc, sign(0) = 0; the formula is
+ *       applied as written to every code, including the unused 2^B-1;
+ *   - q(t) = a t + b t^2 + c t^3 with c = 1 - a - b  [CQ core];
+ *   - w = s * sign(k) * q(t), s FP32, a and b FP16  [CQ core];
+ *   - codes are packed LSB-first: code k of a row occupies bits
+ *     [k*B, k*B+B) of the row's byte stream, bit j in byte j/8 at bit j%8
+ *     (the article only says "dense, contiguous"  [CQ two]);
+ *   - groups are G consecutive elements along K inside one row; scales are
+ *     float32 [N][K/G]; ab is fp16 [N][K/G][2] holding (a, b).
+ *
+ * Parity pins for every function are in tests/test_oracle_*.py.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+#define CQO_MIDRISE 0
+#define CQO_MIDTREAD 1
+
+/* ------------------------------------------------------------------------ */
+/* IEEE number helpers (written from the binary16 / bfloat16 definitions)    */
+/* ------------------------------------------------------------------------ */
+
+/* binary16 bit pattern -> exact double. */
+double cqo_half_to_double(uint16_t h)
+{
+    int sign = h >> 15;
+    int e = (h >> 10) & 31;
+    int m = h & 1023;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);              /* subnormal: m * 2^-24 */
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + m), e - 25);  /* (1 + m/1024) * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+/* double -> binary16 bit pattern, round to nearest, ties to even. */
+uint16_t cqo_double_to_half(double x)
+{
+    uint16_t sign = (uint16_t)(signbit(x) ? 0x8000 : 0);
+    double ax = fabs(x);
+    if (isnan(x))
+        return 0x7e00;
+    if (ax >= 65520.0)                           /* rounds to infinity */
+        return sign | 0x7c00;
+    if (ax < ldexp(1.0, -14)) {                  /* subnormal range, unit 2^-24 */
+        double q = ax * 16777216.0;              /* exact scaling by 2^24 */
+        double r = nearbyint(q);                 /* default mode: ties to even */
+        return sign | (uint16_t)r;               /* r == 1024 gives min normal */
+    }
+    int e;
+    double f = frexp(ax, &e);                    /* ax = f * 2^e, f in [0.5,1) */
+    /* significand with 11 bits: ax = M * 2^(e-11), M in [1024, 2048) */
+    double M = nearbyint(ldexp(f, 11));
+    if (M == 2048.0) { M = 1024.0; e += 1; }
+    int E = e - 1 + 15;                          /* biased exponent */
+    if (E >= 31)
+        return sign | 0x7c00;
+    return sign | (uint16_t)(E << 10) | (uint16_t)((int)M - 1024);
+}
+
+/* float -> bfloat16 bit pattern, round to nearest, ties to even. */
+uint16_t cqo_float_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu))
+        return 0x7fc0;                           /* quiet NaN */
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+double cqo_bf16_to_double(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Bit stream  [CQ two]: dense B-bit codes, LSB-first inside each row         */
+/* ------------------------------------------------------------------------ */
+
+/* codes[N][K] (one code per byte, each < 2^B) -> packed[N][K*B/8]. */
+void cqo_pack(const uint8_t *codes, int64_t N, int64_t K, int B, uint8_t *packed)
+{
+    int64_t row_bytes = K * B / 8;
+    memset(packed, 0, (size_t)(N * row_bytes));
+    for (int64_t n = 0; n < N; n++) {
+        uint8_t *dst = packed + n * row_bytes;
+        for (int64_t k = 0; k < K; k++) {
+            unsigned u = codes[n * K + k];
+            for (int j = 0; j < B; j++) {
+                int64_t bit = k * B + j;
+                if ((u >> j) & 1u)
+                    dst[bit / 8] |= (uint8_t)(1u << (bit % 8));
+            }
+        }
+    }
+}
+
+/* packed[N][K*B/8] -> codes[N][K]. */
+void cqo_unpack(const uint8_t *packed, int64_t N, int64_t K, int B, uint8_t *codes)
+{
+    int64_t row_bytes = K * B / 8;
+    for (int64_t n = 0; n < N; n++) {
+        const uint8_t *src = packed + n * row_bytes;
+        for (int64_t k = 0; k < K; k++) {
+            unsigned u = 0;
+            for (int j = 0; j < B; j++) {
+                int64_t bit = k * B + j;
+                u |= (unsigned)((src[bit / 8] >> (bit % 8)) & 1u) << j;
+            }
+            codes[n * K + k] = (uint8_t)u;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Level math  [CQ core]                                                     */
+/* ------------------------------------------------------------------------ */
+
+/* Signed coordinate of code u: returns sign(k) in {-1,0,+1} and t = |k|/Kc. */
+void cqo_coord(int u, int B, int mode, int *sign, double *t)
+{
+    if (mode == CQO_MIDRISE) {
+        double Kc = ((1 << B) - 1) / 2.0;        /* half-integer half-range */
+        double k = (double)u - Kc;               /* never zero */
+        *sign = k > 0 ? 1 : -1;
+        *t = fabs(k) / Kc;
+    } else {
+        int Kc = (1 << (B - 1)) - 1;
+        int k = u - Kc;
+        *sign = (k > 0) - (k < 0);
+        *t = (double)abs(k) / (double)Kc;
+    }
+}
+
+/* q(t) = a t + b t^2 + c t^3, c = 1 - a - b, evaluated term by term in FP64. */
+double cqo_q(double t, double a, double b)
+{
+    double c = 1.0 - a - b;
+    return a * t + b * t * t + c * t * t * t;
+}
+
+/* Reconstructed weight w = s * sign(k) * q(t) in FP64 for code u. */
+double cqo_level(int u, int B, int mode, float s, uint16_t a_h, uint16_t b_h)
+{
+    int sg;
+    double t;
+    cqo_coord(u, B, mode, &sg, &t);
+    double a = cqo_half_to_double(a_h);
+    double b = cqo_half_to_double(b_h);
+    return (double)s * (double)sg * cqo_q(t, a, b);
+}
+
+/* All 2^B levels of one group, in code order. */
+void cqo_levels(int B, int mode, float s, uint16_t a_h, uint16_t b_h, double *out)
+{
+    for (int u = 0; u < (1 << B); u++)
+        out[u] = cqo_level(u, B, mode, s, a_h, b_h);
+}
+
+/*
+ * Exact monotonicity test of q on [0,1] for stored FP16 (a, b): q'(t) =
+ * a + 2 b t + 3 c t^2 > 0 for every t in [0,1] ([CQ core]: "candidates must
+ * satisfy q'(t) > 0 so that levels never cross").  Every FP16 value is an
+ * integer multiple of 2^-24, so A = a*2^24, Bv = b*2^24, C = 2^24 - A - Bv
+ * are integers and the test is done in exact integer arithmetic:
+ *   q'(0) = a > 0,  q'(1) = 3 - 2a - b > 0, and when the parabola 3c t^2 +
+ *   2b t + a has its minimum inside (0,1) (c > 0 and 0 < -b < 3c), the
+ *   minimum a - b^2/(3c) must be > 0, i.e. Bv^2 < 3 A C.
+ * Returns 1 when q is strictly increasing on [0,1].
+ */
+int cqo_is_monotone(uint16_t a_h, uint16_t b_h)
+{
+    double a = cqo_half_to_double(a_h), b = cqo_half_to_double(b_h);
+    if (!isfinite(a) || !isfinite(b))
+        return 0;
+    __int128 A = (__int128)llround(ldexp(a, 24));
+    __int128 Bv = (__int128)llround(ldexp(b, 24));
+    __int128 one = (__int128)1 << 24;
+    __int128 C = one - A - Bv;
+    if (A <= 0)
+        return 0;
+    if (3 * one - 2 * A - Bv <= 0)
+        return 0;
+    if (C > 0 && -Bv > 0 && -Bv < 3 * C) {
+        if (Bv * Bv >= 3 * A * C)
+            return 0;
+    }
+    return 1;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decode  [CQ core] + [CQ fused]                                            */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * packed + scales + ab -> W in three forms: exact FP64 levels (may be NULL),
+ * the FP64 level rounded once to FP32, and that FP32 rounded to BF16.
+ */
+void cqo_decode(const uint8_t *packed, const float *scales, const uint16_t *ab,
+                int64_t N, int64_t K, int B, int G, int mode,
+                double *w64, float *w32, uint16_t *w16)
+{
+    int64_t ng = K / G;
+    uint8_t *codes = (uint8_t *)malloc((size_t)K);
+    for (int64_t n = 0; n < N; n++) {
+        cqo_unpack(packed + n * (K * B / 8), 1, K, B, codes);
+        for (int64_t k = 0; k < K; k++) {
+            int64_t g = k / G;
+            float s = scales[n * ng + g];
+            uint16_t a_h = ab[(n * ng + g) * 2 + 0];
+            uint16_t b_h = ab[(n * ng + g) * 2 + 1];
+            double L = cqo_level(codes[k], B, mode, s, a_h, b_h);
+            float L32 = (float)L;                /* one RNE rounding to FP32 */
+            if (w64) w64[n * K + k] = L;
+            if (w32) w32[n * K + k] = L32;
+            if (w16) w16[n * K + k] = cqo_float_to_bf16(L32);
+        }
+    }
+    free(codes);
+}
+
+/* ------------------------------------------------------------------------ */
+/* GEMM  [CQ fused]: y[m][n] = sum_k x[m][k] * w[n][k], FP64                 */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t *x; int64_t M;
+    const uint8_t *packed; const float *scales; const uint16_t *ab;
+    int64_t N, K; int B, G, mode;
+    double *y, *bound;
+    int64_t n0, n1;
+} gemm_job;
+
+static void *gemm_worker(void *p)
+{
+    gemm_job *j = (gemm_job *)p;
+    double *wrow = (double *)malloc((size_t)j->K * sizeof(double));
+    int64_t rb = j->K * j->B / 8, ng = j->K / j->G;
+    for (int64_t n = j->n0; n < j->n1; n++) {
+        /* this row's exact levels */
+        cqo_decode(j->packed + n * rb, j->scales + n * ng, j->ab + n * ng * 2,
+                   1, j->K, j->B, j->G, j->mode, wrow, NULL, NULL);
+        for (int64_t m = 0; m < j->M; m++) {
+            double acc = 0.0, bnd = 0.0;
+            for (int64_t k = 0; k < j->K; k++) {
+                double xv = cqo_bf16_to_double(j->x[m * j->K + k]);
+                acc += xv * wrow[k];
+                bnd += fabs(xv * wrow[k]);
+            }
+            j->y[m * j->N + n] = acc;
+            if (j->bound)
+                j->bound[m * j->N + n] = bnd;
+        }
+    }
+    free(wrow);
+    return NULL;
+}
+
+int cqo_num_threads(int requested)
+{
+    if (requested > 0)
+        return requested;
+    long c = sysconf(_SC_NPROCESSORS_ONLN);
+    return c > 0 ? (int)c : 1;
+}
+
+/*
+ * x: bf16 [M][K]; W given packed.  y and bound: double [M][N], where
+ * bound[m][n] = sum_k |x[m][k] * w[n][k]| (the scale of the tolerance).
+ * Rows of W are split across threads; each output is one plain sequential
+ * sum over k.
+ */
+void cqo_gemm(const uint16_t *x, int64_t M, const uint8_t *packed, const float *scales,
+              const uint16_t *ab, int64_t N, int64_t K, int B, int G, int mode,
+              double *y, double *bound, int nthreads)
+{
+    int T = cqo_num_threads(nthreads);
+    if (T > N) T = (int)(N > 0 ? N : 1);
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * T);
+    gemm_job *jobs = (gemm_job *)malloc(sizeof(gemm_job) * T);
+    for (int i = 0; i < T; i++) {
+        gemm_job j = {x, M, packed, scales, ab, N, K, B, G, mode, y, bound,
+                      N * i / T, N * (i + 1) / T};
+        jobs[i] = j;
+        pthread_create(&th[i], NULL, gemm_worker, &jobs[i]);
+    }
+    for (int i = 0; i < T; i++)
+        pthread_join(th[i], NULL);
+    free(th);
+    free(jobs);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Data-free group fitter  [CQ fit]                                          */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Nearest level: the index u of the level closest to v, ties to the lower
+ * code.  Levels are sorted ascending (q is increasing and the grid is
+ * sign-symmetric), so a binary search finds the bracketing pair.
+ */
+int cqo_nearest(const double *lv, int nlev, double v)
+{
+    int lo = 0, hi = nlev - 1;
+    if (v <= lv[0]) return 0;
+    if (v >= lv[hi]) return hi;
+    while (hi - lo > 1) {                       /* invariant lv[lo] < v < lv[hi] */
+        int mid = (lo + hi) / 2;
+        if (lv[mid] <= v) lo = mid; else hi = mid;
+    }
+    if (lv[lo] == v) return lo;
+    return (v - lv[lo] <= lv[hi] - v) ? lo : hi;
+}
+
+/* Linear-scan nearest level (brute force, used by the tests as a pin). */
+int cqo_nearest_bruteforce(const double *lv, int nlev, double v)
+{
+    int best = 0;
+    double bd = fabs(v - lv[0]);
+    for (int u = 1; u < nlev; u++) {
+        double d = fabs(v - lv[u]);
+        if (d < bd) { bd = d; best = u; }
+    }
+    return best;
+}
+
+typedef struct {
+    /* candidate grid */
+    int na, nb, nalpha;
+    const double *a_grid, *b_grid, *alpha_grid;
+    int uniform_only;          /* 1: only (a,b) = (1,0)  -> optimal clipped INT */
+} fit_cfg;
+
+/* Number of codes a grid mode uses: 2^B (midrise) or 2^B - 1 (midtread). */
+static int used_levels(int B, int mode)
+{
+    return mode == CQO_MIDRISE ? (1 << B) : (1 << B) - 1;
+}
+
+/* SSE of group w[G] under (s, a_h, b_h); codes written when out != NULL. */
+static double group_sse(const double *w, int G, int B, int mode, float s,
+                        uint16_t a_h, uint16_t b_h, uint8_t *codes_out, int *clipped)
+{
+    double lv[256];
+    int nl = used_levels(B, mode);
+    cqo_levels(B, mode, s, a_h, b_h, lv);
+    double sse = 0.0;
+    int clip = 0;
+    for (int i = 0; i < G; i++) {
+        int u = cqo_nearest(lv, nl, w[i]);
+        double e = w[i] - lv[u];
+        sse += e * e;
+        if (fabs(w[i]) > (double)s) clip++;
+        if (codes_out) codes_out[i] = (uint8_t)u;
+    }
+    if (clipped) *clipped = clip;
+    return sse;
+}
+
+/*
+ * Fit one group, following the article's steps [CQ fit]:
+ *   (1) the group is given;
+ *   (2) search monotone (a, b) candidates -- the uniform point (1, 0) is
+ *       always a candidate;
+ *   (3) jointly search the scale / clipping threshold s = alpha * max|w|;
+ *   (4) assign every weight to its nearest reconstruction level;
+ *   (5) cast a, b to FP16 and keep s in FP32, then recompute the codes and
+ *       the error with the stored values.
+ * The objective is the group's squared error.  Ties keep the earliest
+ * candidate in enumeration order: (1,0) first, then the (a,b) grid in order,
+ * and for each (a,b) alpha ascending.
+ * Outputs: codes[G], s, a_h, b_h; return value = SSE with stored values.
+ */
+static double fit_group(const double *w, int G, int B, int mode, const fit_cfg *cfg,
+                        uint8_t *codes, float *s_out, uint16_t *a_out, uint16_t *b_out,
+                        int *clipped)
+{
+    double mx = 0.0;
+    for (int i = 0; i < G; i++)
+        if (fabs(w[i]) > mx) mx = fabs(w[i]);
+    if (mx == 0.0) {                             /* all-zero group */
+        *s_out = 0.0f;
+        *a_out = cqo_double_to_half(1.0);
+        *b_out = cqo_double_to_half(0.0);
+        return group_sse(w, G, B, mode, 0.0f, *a_out, *b_out, codes, clipped);
+    }
+    double best = INFINITY;
+    double best_a = 1.0, best_b = 0.0;
+    float best_s = (float)mx;
+    int ncand = cfg->uniform_only ? 1 : 1 + cfg->na * cfg->nb;
+    for (int c = 0; c < ncand; c++) {
+        double a, b;
+        if (c == 0) { a = 1.0; b = 0.0; }
+        else {
+            a = cfg->a_grid[(c - 1) / cfg->nb];
+            b = cfg->b_grid[(c - 1) % cfg->nb];
+            if (a == 1.0 && b == 0.0) continue;
+        }
+        uint16_t a_h = cqo_double_to_half(a), b_h = cqo_double_to_half(b);
+        if (!cqo_is_monotone(a_h, b_h)) continue;
+        for (int ia = 0; ia < cfg->nalpha; ia++) {
+            float s = (float)(cfg->alpha_grid[ia] * mx);
+            double e = group_sse(w, G, B, mode, s, a_h, b_h, NULL, NULL);
+            if (e < best) { best = e; best_a = a; best_b = b; best_s = s; }
+        }
+    }
+    /* step (5): FP16 a, b and FP32 s, then codes and error recomputed */
+    *a_out = cqo_double_to_half(best_a);
+    *b_out = cqo_double_to_half(best_b);
+    *s_out = best_s;
+    return group_sse(w, G, B, mode, best_s, *a_out, *b_out, codes, clipped);
+}
+
+typedef struct {
+    const double *w; int64_t ngroups; int G, B, mode;
+    const fit_cfg *cfg;
+    uint8_t *codes; float *s; uint16_t *ab; double *sse; int32_t *clipped;
+    int64_t g0, g1;
+} fit_job;
+
+static void *fit_worker(void *p)
+{
+    fit_job *j = (fit_job *)p;
+    for (int64_t g = j->g0; g < j->g1; g++) {
+        int clip = 0;
+        double e = fit_group(j->w + g * j->G, j->G, j->B, j->mode, j->cfg,
+                             j->codes + g * j->G, &j->s[g], &j->ab[2 * g],
+                             &j->ab[2 * g + 1], &clip);
+        j->sse[g] = e;
+        j->clipped[g] = clip;
+    }
+    return NULL;
+}
+
+/*
+ * Fit ngroups independent groups of G weights (w is [ngroups][G]).
+ * Outputs per group: codes [ngroups][G], s [ngroups], ab [ngroups][2] (fp16
+ * bits), sse [ngroups], clipped [ngroups] (count of |w| > s).
+ */
+void cqo_fit(const double *w, int64_t ngroups, int G, int B, int mode,
+             const double *a_grid, int na, const double *b_grid, int nb,
+             const double *alpha_grid, int nalpha, int uniform_only,
+             uint8_t *codes, float *s, uint16_t *ab, double *sse, int32_t *clipped,
+             int nthreads)
+{
+    fit_cfg cfg = {na, nb, nalpha, a_grid, b_grid, alpha_grid, uniform_only};
+    int T = cqo_num_threads(nthreads);
+    if (T > ngroups) T = (int)(ngroups > 0 ? ngroups : 1);
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * T);
+    fit_job *jobs = (fit_job *)malloc(sizeof(fit_job) * T);
+    for (int i = 0; i < T; i++) {
+        fit_job j = {w, ngroups, G, B, mode, &cfg, codes, s, ab, sse, clipped,
+                     ngroups * i / T, ngroups * (i + 1) / T};
+        jobs[i] = j;
+        pthread_create(&th[i], NULL, fit_worker, &jobs[i]);
+    }
+    for (int i = 0; i < T; i++)
+        pthread_join(th[i], NULL);
+    free(th);
+    free(jobs);
+}
+
+/*
+ * Exact minimum SSE of ANY nlev-level scalar quantizer of the n values v
+ * (the free-codebook / Lloyd-Max side of the error bound in [CQ two]).
+ * Optimal 1-D clustering by dynamic programming over the sorted values
+ * (Bellman; Wang & Song, "Ckmeans.1d.dp", 2011): cost(i, j) is the SSE of
+ * values i..j around their mean, D[l][j] = min_i D[l-1][i-1] + cost(i, j).
+ */
+static int cmp_double(const void *a, const void *b)
+{
+    double x = *(const double *)a, y = *(const double *)b;
+    return (x > y) - (x < y);
+}
+
+double cqo_optimal_sse(const double *v_in, int n, int nlev)
+{
+    double *v = (double *)malloc(sizeof(double) * n);
+    memcpy(v, v_in, sizeof(double) * n);
+    qsort(v, n, sizeof(double), cmp_double);
+    double *S1 = (double *)calloc(n + 1, sizeof(double));
+    double *S2 = (double *)calloc(n + 1, sizeof(double));
+    for (int i = 0; i < n; i++) {
+        S1[i + 1] = S1[i] + v[i];
+        S2[i + 1] = S2[i] + v[i] * v[i];
+    }
+    if (nlev > n) nlev = n;
+    double *D = (double *)malloc(sizeof(double) * (n + 1) * (nlev + 1));
+#define DD(l, j) D[(l) * (n + 1) + (j)]
+    for (int j = 0; j <= n; j++) DD(0, j) = (j == 0) ? 0.0 : INFINITY;
+    for (int l = 1; l <= nlev; l++) {
+        DD(l, 0) = 0.0;
+        for (int j = 1; j <= n; j++) {
+            double best = INFINITY;
+            for (int i = l; i <= j; i++) {     /* last cluster = v[i-1 .. j-1] */
+                double cnt = j - i + 1;
+                double s1 = S1[j] - S1[i - 1], s2 = S2[j] - S2[i - 1];
+                double cost = s2 - s1 * s1 / cnt;
+                if (cost < 0) cost = 0;
+                double c = DD(l - 1, i - 1) + cost;
+                if (c < best) best = c;
+            }
+            DD(l, j) = best;
+        }
+    }
+    double r = DD(nlev, n);
+#undef DD
+    free(D); free(S1); free(S2); free(v);
+    return r;
+}
