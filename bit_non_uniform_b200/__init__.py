@@ -1,0 +1,214 @@
+"""Python binding of libcq, the B200 CubicQuant weight-only GEMM library.
+
+This module only marshals arguments: every step of the computation runs in
+the CUDA kernels of ``libcq.so`` (built in-tree by ``build.py``).  There is
+no CPU fallback; if the library is missing or a call fails, an exception is
+raised.  PyTorch is used for device memory and streams.
+
+The calls mirror ``include/cq.h``:
+
+* ``cq_pack(codes, B)``                         -> packed [N][K*B/8] uint8
+* ``cq_decode(packed, scales, ab, K, B, G)``    -> W [N][K] (float32 / bfloat16)
+* ``cq_gemm(x, packed, scales, ab, N, K, B, G)`` -> y [M][N] (or [M][N/2])
+* ``cq_moe_grouped_gemm(tokens, topk_ids, ...)`` -> per-route / combined outputs
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libcq.so")
+
+MIDRISE, MIDTREAD = 0, 1
+F32, BF16 = 0, 1
+EPI_NONE, EPI_SWIGLU = 0, 1
+
+_STATUS = {
+    0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA runtime error",
+    4: "a bounded device wait ran out", 5: "workspace missing or too small",
+}
+
+
+class CQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: libcq status {status} ({_STATUS.get(status, '?')})")
+        self.status = status
+
+
+_lib = None
+
+
+class MatrixDesc(ctypes.Structure):
+    _fields_ = [("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("ab", ctypes.c_void_p), ("B", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class ExpertDesc(ctypes.Structure):
+    _fields_ = [("gate_up", MatrixDesc), ("down", MatrixDesc)]
+
+
+def lib():
+    """Load libcq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"libcq.so not found at {LIB_PATH}; build it with "
+            "`python -m bit_non_uniform_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i64, i32, sz, u64 = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t,
+                            ctypes.c_uint64)
+    sigs = {
+        "cq_version": (i32, []),
+        "cq_status_string": (ctypes.c_char_p, [i32]),
+        "cq_pack": (i32, [P, i64, i64, i32, P, P]),
+        "cq_decode": (i32, [P, P, P, i64, i64, i32, i32, i32, i32, P, P]),
+        "cq_gemm_workspace_size": (sz, [i64, i64, i64, i32, i32, i32]),
+        "cq_gemm": (i32, [P, i64, P, P, P, i64, i64, i32, i32, i32, i32, i32, P, P, sz, P]),
+        "cq_moe_workspace_size": (sz, [i64, i32, i32, i64, i64, i32]),
+        "cq_moe_grouped_gemm": (i32, [P, i64, P, P, i32, i32, P, i64, i64, i32, i32, i32,
+                                      P, P, P, sz, P]),
+        "cq_get_device_error": (i32, [P, ctypes.POINTER(ctypes.c_int)]),
+        "cq_test_gemm_bounded": (i32, [P, i64, P, P, P, i64, i64, i32, i32, P, P, sz, u64,
+                                       i32, P]),
+    }
+    for name, (res, args) in sigs.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise CQError(st, where)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libcq works on CUDA tensors only")
+
+
+def version() -> int:
+    return int(lib().cq_version())
+
+
+def cq_pack(codes: torch.Tensor, B: int, out: torch.Tensor | None = None, stream=None):
+    """codes uint8 [N][K] (CUDA) -> packed uint8 [N][K*B/8]."""
+    _need_cuda(codes)
+    codes = codes.contiguous()
+    N, K = codes.shape
+    if out is None:
+        out = torch.empty((N, K * B // 8), dtype=torch.uint8, device=codes.device)
+    _check(lib().cq_pack(_ptr(codes), N, K, B, _ptr(out), _stream(stream)), "cq_pack")
+    return out
+
+
+def cq_decode(packed, scales, ab, K: int, B: int, G: int, mode: int = MIDRISE,
+              out_dtype: int = F32, stream=None):
+    """Decode packed codes + (s, a, b) into W [N][K] (float32 or bfloat16)."""
+    _need_cuda(packed, scales, ab)
+    N = packed.shape[0]
+    dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+    W = torch.empty((N, K), dtype=dt, device=packed.device)
+    _check(lib().cq_decode(_ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G, mode, out_dtype,
+                           _ptr(W), _stream(stream)), "cq_decode")
+    return W
+
+
+def gemm_workspace_size(M, N, K, B, G, epilogue=EPI_NONE) -> int:
+    return int(lib().cq_gemm_workspace_size(M, N, K, B, G, epilogue))
+
+
+def gemm_workspace(M, N, K, B, G, epilogue=EPI_NONE, device="cuda"):
+    """A zero-initialised workspace buffer for cq_gemm."""
+    n = gemm_workspace_size(M, N, K, B, G, epilogue)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def cq_gemm(x, packed, scales, ab, N: int, K: int, B: int, G: int, mode: int = MIDRISE,
+            epilogue: int = EPI_NONE, out_dtype: int = F32, workspace=None, out=None,
+            stream=None):
+    """y = x W^T with W given packed; x bfloat16 [M][K]."""
+    _need_cuda(x, packed, scales, ab)
+    assert x.dtype == torch.bfloat16 and x.is_contiguous()
+    M = x.shape[0]
+    ncol = N // 2 if epilogue == EPI_SWIGLU else N
+    if out is None:
+        dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+        out = torch.empty((M, ncol), dtype=dt, device=x.device)
+    if workspace is None:
+        workspace = gemm_workspace(M, N, K, B, G, epilogue, x.device)
+    _check(lib().cq_gemm(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G, mode,
+                         epilogue, out_dtype, _ptr(out), _ptr(workspace),
+                         workspace.numel() * workspace.element_size(), _stream(stream)),
+           "cq_gemm")
+    return out
+
+
+def moe_workspace_size(T, k, E, H, I, G) -> int:
+    return int(lib().cq_moe_workspace_size(T, k, E, H, I, G))
+
+
+def expert_table(experts, device="cuda"):
+    """Pack a list of per-expert dicts (gate_up / down packed, scales, ab, B)
+    into the device array of cq_expert_desc that cq_moe_grouped_gemm reads."""
+    arr = (ExpertDesc * len(experts))()
+    for e, ex in enumerate(experts):
+        for fld, key in (("gate_up", "gu"), ("down", "dn")):
+            d = getattr(arr[e], fld)
+            d.packed = ex[f"packed_{key}"].data_ptr()
+            d.scales = ex[f"scales_{key}"].data_ptr()
+            d.ab = ex[f"ab_{key}"].data_ptr()
+            d.B = int(ex[f"B_{key}"])
+            d.reserved = 0
+    raw = bytes(arr)
+    host = torch.frombuffer(bytearray(raw), dtype=torch.uint8)
+    return host.to(device)
+
+
+def cq_moe_grouped_gemm(tokens, topk_ids, topk_w, expert_descs, E: int, H: int, I: int,
+                        G: int, mode: int = MIDRISE, out_dtype: int = F32,
+                        route_out=True, combine=True, workspace=None, stream=None):
+    """Routed-expert FFN of one MoE layer.  Returns (route_out, out)."""
+    _need_cuda(tokens, topk_ids, expert_descs)
+    T, k = topk_ids.shape
+    ro = None
+    if route_out is True:
+        ro = torch.empty((T * k, H), dtype=torch.float32, device=tokens.device)
+    elif route_out is not None and route_out is not False:
+        ro = route_out
+    out = None
+    if combine:
+        dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+        out = torch.empty((T, H), dtype=dt, device=tokens.device)
+    if workspace is None:
+        n = moe_workspace_size(T, k, E, H, I, G)
+        workspace = torch.zeros(max(n, 16), dtype=torch.uint8, device=tokens.device)
+    _check(lib().cq_moe_grouped_gemm(
+        _ptr(tokens), T, _ptr(topk_ids), _ptr(topk_w) if topk_w is not None else None, k, E,
+        _ptr(expert_descs), H, I, G, mode, out_dtype, _ptr(ro), _ptr(out), _ptr(workspace),
+        workspace.numel(), _stream(stream)), "cq_moe_grouped_gemm")
+    return ro, out
+
+
+def device_error(stream=None) -> tuple[int, int]:
+    """(status, site) of the device error word; clears it."""
+    site = ctypes.c_int(0)
+    st = lib().cq_get_device_error(_stream(stream), ctypes.byref(site))
+    return int(st), int(site.value)

@@ -1,0 +1,150 @@
+// cq_gemm.cu -- host side of cq_gemm: argument checks, work partition,
+// activation tensor map and the engine launch.
+#include <cuda_runtime.h>
+
+#include "cq.h"
+#include "cq_engine.cuh"
+#include "cq_host.h"
+
+namespace cq {
+
+static int pick_nt(int64_t M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  return 128;
+}
+
+struct GemmPlan {
+  int NT, n_tt, n_rt, spt, tiles, P;
+  size_t ws_counter_bytes, ws_partial_bytes;
+};
+
+static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int epilogue, int sms) {
+  GemmPlan g;
+  g.NT = pick_nt(M);
+  g.n_tt = static_cast<int>((M + g.NT - 1) / g.NT);
+  g.n_rt = epilogue == CQ_EPI_SWIGLU ? static_cast<int>(N / kRows)
+                                     : static_cast<int>((N + kRows - 1) / kRows);
+  g.spt = static_cast<int>(K / kSlice);
+  g.tiles = g.n_rt * g.n_tt;
+  const int64_t W = static_cast<int64_t>(g.tiles) * g.spt;
+  g.P = static_cast<int>(W < sms ? W : sms);
+  g.ws_counter_bytes = ((static_cast<size_t>(g.tiles) * sizeof(int) + 255) / 256) * 256;
+  g.ws_partial_bytes = static_cast<size_t>(2) * g.P * g.NT * kRows * sizeof(float);
+  return g;
+}
+
+template <int NT>
+static int launch_engine(const EngineParams& p, const CUtensorMap& map, cudaStream_t s) {
+  using C = EngineCfg<NT>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(engine_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM) != cudaSuccess)
+      return CQ_ERR_CUDA;
+    attr_set = true;
+  }
+  engine_kernel<NT><<<p.P, kThreads, C::SMEM, s>>>(p, map);
+  return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* scales,
+              const uint16_t* ab, int64_t N, int64_t K, int B, int G, int grid_mode,
+              int epilogue, int out_dtype, void* y, void* workspace, size_t ws_bytes,
+              cudaStream_t stream, uint64_t timeout_ns, int debug_skip) {
+  int st = validate_matrix(packed, scales, ab, N, K, B, G, grid_mode);
+  if (st != CQ_OK) return st;
+  if (M < 0) return CQ_ERR_INVALID_ARG;
+  if (epilogue != CQ_EPI_NONE && epilogue != CQ_EPI_SWIGLU) return CQ_ERR_INVALID_ARG;
+  if (out_dtype != CQ_DTYPE_F32 && out_dtype != CQ_DTYPE_BF16) return CQ_ERR_INVALID_ARG;
+  if (epilogue == CQ_EPI_SWIGLU && N % kRows != 0) return CQ_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return CQ_OK;
+  if (K == 0) return CQ_ERR_UNSUPPORTED;
+  if (!x || !y) return CQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16)) return CQ_ERR_UNSUPPORTED;
+  if (M > (int64_t)1 << 24) return CQ_ERR_UNSUPPORTED;
+  const int sms = num_sms();
+  if (sms <= 0) return CQ_ERR_CUDA;
+  const GemmPlan g = plan_gemm(M, N, K, epilogue, sms);
+  const size_t need = g.ws_counter_bytes + g.ws_partial_bytes;
+  if (ws_bytes < need || (need && !workspace)) return CQ_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return CQ_ERR_UNSUPPORTED;
+
+  CUtensorMap map;
+  st = encode_bf16_rows_sw128(&map, x, M, K, g.NT);
+  if (st != CQ_OK) return st;
+
+  EngineParams p = {};
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.G = G;
+  p.mode = grid_mode;
+  p.epilogue = epilogue;
+  p.out_bf16 = out_dtype == CQ_DTYPE_BF16;
+  p.n_rt = g.n_rt;
+  p.spt = g.spt;
+  p.num_tiles = g.tiles;
+  p.P = g.P;
+  p.mat.packed = packed;
+  p.mat.scales = scales;
+  p.mat.ab = reinterpret_cast<const uint32_t*>(ab);
+  p.mat.B = B;
+  p.M = static_cast<int>(M);
+  p.n_tt = g.n_tt;
+  p.y = y;
+  p.ldy = epilogue == CQ_EPI_SWIGLU ? N / 2 : N;
+  p.counter = reinterpret_cast<int*>(workspace);
+  p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + g.ws_counter_bytes);
+  p.timeout_ns = timeout_ns;
+  p.debug_skip_first_stage = debug_skip;
+
+  switch (g.NT) {
+    case 16: return launch_engine<16>(p, map, stream);
+    case 32: return launch_engine<32>(p, map, stream);
+    case 64: return launch_engine<64>(p, map, stream);
+    default: return launch_engine<128>(p, map, stream);
+  }
+}
+
+size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int epilogue, int sms) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % kSlice != 0) return 0;
+  const GemmPlan g = plan_gemm(M, N, K, epilogue, sms);
+  return g.ws_counter_bytes + g.ws_partial_bytes;
+}
+
+}  // namespace cq
+
+using namespace cq;
+
+static constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;   // 2 s per wait
+
+extern "C" size_t cq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int B, int G,
+                                         int epilogue) {
+  (void)B;
+  (void)G;
+  int sms = num_sms();
+  if (sms <= 0) sms = 148;
+  return gemm_workspace_size(M, N, K, epilogue, sms);
+}
+
+extern "C" int cq_gemm(const uint16_t* x, int64_t M, const uint8_t* packed, const float* scales,
+                       const uint16_t* ab, int64_t N, int64_t K, int B, int G, int grid_mode,
+                       int epilogue, int out_dtype, void* y, void* workspace, size_t ws_bytes,
+                       void* stream) {
+  return gemm_impl(x, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype, y,
+                   workspace, ws_bytes, static_cast<cudaStream_t>(stream), kDefaultTimeoutNs, 0);
+}
+
+// Test hook (not part of the public header): run cq_gemm with a chosen wait
+// limit and, optionally, with the first stage load withheld so that the
+// bounded waits run out; the caller then reads CQ_ERR_TIMEOUT from
+// cq_get_device_error().
+extern "C" CQ_API int cq_test_gemm_bounded(const uint16_t* x, int64_t M, const uint8_t* packed,
+                                    const float* scales, const uint16_t* ab, int64_t N, int64_t K,
+                                    int B, int G, void* y, void* workspace, size_t ws_bytes,
+                                    uint64_t timeout_ns, int skip_first_stage, void* stream) {
+  return gemm_impl(x, M, packed, scales, ab, N, K, B, G, CQ_GRID_MIDRISE, CQ_EPI_NONE,
+                   CQ_DTYPE_F32, y, workspace, ws_bytes, static_cast<cudaStream_t>(stream),
+                   timeout_ns, skip_first_stage);
+}

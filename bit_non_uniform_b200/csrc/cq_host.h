@@ -1,0 +1,78 @@
+// cq_host.h -- host-side argument validation and TMA descriptor encoding
+// shared by the libcq entry points.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "cq.h"
+
+namespace cq {
+
+inline bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+// Checks shared by every call that reads a packed CubicQuant matrix.
+inline int validate_matrix(const uint8_t* packed, const float* scales, const uint16_t* ab,
+                           int64_t N, int64_t K, int B, int G, int grid_mode) {
+  if (N < 0 || K < 0 || G <= 0) return CQ_ERR_INVALID_ARG;
+  if (grid_mode != CQ_GRID_MIDRISE && grid_mode != CQ_GRID_MIDTREAD) return CQ_ERR_INVALID_ARG;
+  if (B < 2 || B > 4) return CQ_ERR_UNSUPPORTED;
+  if (G % 128 != 0 || K % G != 0) return CQ_ERR_UNSUPPORTED;
+  if (N * K == 0) return CQ_OK;
+  if (!packed || !scales || !ab) return CQ_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(scales, 4) || !aligned(ab, 4)) return CQ_ERR_UNSUPPORTED;
+  if (K > (int64_t)1 << 30 || N > (int64_t)1 << 30) return CQ_ERR_UNSUPPORTED;
+  return CQ_OK;
+}
+
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Tensor map over a row-major bf16 matrix [rows][cols] loaded as boxes of
+// 64 columns (128 bytes) x box_rows rows with the 128-byte swizzle.  Rows
+// past `rows` read as zero.
+inline int encode_bf16_rows_sw128(CUtensorMap* map, const void* base, int64_t rows,
+                                  int64_t cols, int box_rows) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return CQ_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CQ_OK : CQ_ERR_CUDA;
+}
+
+inline int num_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return sms;
+}
+
+}  // namespace cq

@@ -1,0 +1,177 @@
+/*
+ * cq.h -- C ABI of libcq, the B200 (sm_100a) CubicQuant weight-only GEMM
+ * library.
+ *
+ * The method (ModelScope article "CubicQuant：用三次曲线重塑低比特量化，Kimi
+ * K3 2.5Bit 模型首发实践", cited as [CQ]) stores each weight as a B-bit code
+ * u, packed densely, in groups of G weights that carry an FP32 scale s and
+ * two FP16 shape parameters a, b (c = 1 - a - b is derived).  A code
+ * decodes to
+ *         w = s * sign(k) * q(t),   q(t) = a t + b t^2 + c t^3,
+ * with k the signed integer coordinate of u and t = |k| / Kc its normalised
+ * magnitude ([CQ] section "CubicQuant 核心：把直线网格“掰弯”").  The article's
+ * code-to-coordinate formula was lost in extraction; this library fixes
+ *   CQ_GRID_MIDRISE  (default): Kc = (2^B-1)/2, k = u - Kc, t = |k|/Kc;
+ *   CQ_GRID_MIDTREAD          : Kc = 2^(B-1)-1, k = u - Kc, t = |k|/Kc,
+ *                               sign(0) = 0 (code 2^B-1 is decoded by the
+ *                               same formula; fitters never emit it).
+ * With a = 1, b = 0 both give the symmetric uniform integer grid.
+ *
+ * Data layout (all row-major, all buffers owned by the caller):
+ *   W      logical [N][K] weights; groups are G consecutive K-elements.
+ *   packed uint8 [N][K*B/8]: code (n,k) occupies bits [k*B, k*B+B) of row n's
+ *          byte stream, least significant bit first ([CQ] only says the
+ *          stream is dense and contiguous, section "为什么只用两个形状参数？").
+ *   scales float [N][K/G]                    -- s per group
+ *   ab     uint16 (IEEE binary16) [N][K/G][2] -- (a, b) per group
+ *   x      uint16 (bfloat16) [M][K] activations
+ *   y      [M][N] (or [M][N/2] with CQ_EPI_SWIGLU), float or bfloat16
+ * Storage per weight is B + 64/G bits ([CQ] section "存储开销是透明的").
+ *
+ * Conventions:
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise.
+ *   - Every call is asynchronous on the given cudaStream_t (passed as void*,
+ *     NULL = legacy default stream) and returns a cq_status.  Arguments are
+ *     validated on the host before anything is launched; on error nothing
+ *     is launched and no output is touched.
+ *   - Supported: B in {2,3,4}; G a multiple of 128; K a multiple of G;
+ *     N >= 1; packed / x / y / workspace 16-byte aligned; scales and ab
+ *     4-byte aligned.
+ *   - The library allocates no memory.  Calls that need scratch take a
+ *     caller-provided workspace whose size is given by the matching
+ *     *_workspace_size() query.
+ *   - Device-side waits are bounded; a wait that runs out records an error
+ *     that cq_get_device_error() reports as CQ_ERR_TIMEOUT.
+ */
+#ifndef CQ_H_
+#define CQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CQ_API __attribute__((visibility("default")))
+#else
+#define CQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CQ_OK = 0,
+    CQ_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad enum   */
+    CQ_ERR_UNSUPPORTED = 2,  /* B, G, K, N or alignment not supported  */
+    CQ_ERR_CUDA = 3,         /* a CUDA runtime call failed             */
+    CQ_ERR_TIMEOUT = 4,      /* a bounded device wait ran out          */
+    CQ_ERR_WORKSPACE = 5     /* workspace missing or too small         */
+} cq_status;
+
+enum { CQ_GRID_MIDRISE = 0, CQ_GRID_MIDTREAD = 1 };
+enum { CQ_DTYPE_F32 = 0, CQ_DTYPE_BF16 = 1 };
+enum { CQ_EPI_NONE = 0, CQ_EPI_SWIGLU = 1 };
+
+/* Library version as 10000*major + 100*minor + patch. */
+CQ_API int cq_version(void);
+
+/* Static English description of a cq_status value. */
+CQ_API const char *cq_status_string(int status);
+
+/*
+ * cq_pack -- pack one code per byte into the dense LSB-first bit stream.
+ *   codes  uint8 [N][K], each < 2^B (higher bits are ignored)
+ *   packed uint8 [N][K*B/8] (output)
+ * Requires K*B % 8 == 0.  [CQ] "为什么只用两个形状参数？": codes remain an
+ * ordinary 1-8 bit scalar stream that can be packed contiguously.
+ */
+CQ_API int cq_pack(const uint8_t *codes, int64_t N, int64_t K, int B, uint8_t *packed,
+            void *stream);
+
+/*
+ * cq_decode -- expand packed codes and group parameters into weights.
+ *   out_dtype CQ_DTYPE_F32: W_out float [N][K], each element the level
+ *             s*sign(k)*q(t) evaluated in FP64 and rounded once to FP32;
+ *   out_dtype CQ_DTYPE_BF16: W_out bfloat16 [N][K], that FP32 value rounded
+ *             to nearest-even BF16.
+ * [CQ] "CubicQuant 核心" (reconstruction); this is the parity tool, the GEMM
+ * never materialises W ([CQ] "压缩权重必须“边解码、边计算”").
+ */
+CQ_API int cq_decode(const uint8_t *packed, const float *scales, const uint16_t *ab,
+              int64_t N, int64_t K, int B, int G, int grid_mode, int out_dtype,
+              void *W_out, void *stream);
+
+/*
+ * cq_gemm -- y[m][n] = sum_k x[m][k] * w[n][k] with FP32 accumulation, the
+ * weights decoded tile by tile on chip (A16 path, [CQ] "一份 checkpoint，同时
+ * 服务 A16 与 Dynamic A8" and "压缩权重必须“边解码、边计算”").
+ *   x          bfloat16 [M][K]; M >= 0 (M == 0 is a no-op)
+ *   epilogue   CQ_EPI_NONE: y [M][N];
+ *              CQ_EPI_SWIGLU: rows [0,N/2) are gate, rows [N/2,N) are up,
+ *              y[m][j] = silu(g) * u with silu(g) = g / (1 + exp(-g)),
+ *              y is [M][N/2]; requires N % 128 == 0.
+ *   out_dtype  CQ_DTYPE_F32 or CQ_DTYPE_BF16
+ *   workspace  device scratch of at least cq_gemm_workspace_size(...) bytes
+ *              (may be NULL when that size is 0).  Its first bytes hold
+ *              counters that must be zero before the first call that uses
+ *              the buffer; every completed call leaves them zero again.
+ * Calls that share one workspace must not overlap on the GPU.
+ */
+CQ_API size_t cq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int B, int G,
+                              int epilogue);
+CQ_API int cq_gemm(const uint16_t *x, int64_t M, const uint8_t *packed, const float *scales,
+            const uint16_t *ab, int64_t N, int64_t K, int B, int G, int grid_mode,
+            int epilogue, int out_dtype, void *y, void *workspace, size_t ws_bytes,
+            void *stream);
+
+/*
+ * One quantized matrix as seen by the grouped MoE call (device array).
+ */
+typedef struct {
+    const uint8_t *packed;   /* [rows][cols*B/8]        */
+    const float *scales;     /* [rows][cols/G]          */
+    const uint16_t *ab;      /* [rows][cols/G][2] fp16  */
+    int32_t B;               /* 2, 3 or 4               */
+    int32_t reserved;        /* must be 0               */
+} cq_matrix_desc;
+
+typedef struct {
+    cq_matrix_desc gate_up;  /* [2I][H]: gate rows [0,I), up rows [I,2I) */
+    cq_matrix_desc down;     /* [H][I]                                    */
+} cq_expert_desc;
+
+/*
+ * cq_moe_grouped_gemm -- the routed-expert FFN of one MoE layer, with
+ * per-expert CubicQuant weights (the quantized tensors of [CQ] are the
+ * routed experts, section "先看结论").  For every route r = (t, j):
+ *   e = topk_ids[t][j];  g|u = W_gu[e] x_t;  h = bf16(silu(g) * u);
+ *   y_r = W_dn[e] h  (FP32 accumulation)
+ * and, when out != NULL, out[t] = sum_j topk_w[t][j] * y_(t,j) (j ascending).
+ *   tokens     bfloat16 [T][H]
+ *   topk_ids   int32 [T][k], values in [0, E)
+ *   topk_w     float [T][k] (required when out != NULL)
+ *   experts    device array of E cq_expert_desc
+ *   route_out  float [T*k][H] per-route outputs y_r (may be NULL)
+ *   out        [T][H] combined output in out_dtype (may be NULL)
+ * Requires H and I multiples of G, G % 128 == 0, I % 64 == 0.
+ */
+CQ_API size_t cq_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I, int G);
+CQ_API int cq_moe_grouped_gemm(const uint16_t *tokens, int64_t T, const int32_t *topk_ids,
+                        const float *topk_w, int k, int E,
+                        const cq_expert_desc *experts, int64_t H, int64_t I, int G,
+                        int grid_mode, int out_dtype, void *route_out, void *out,
+                        void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * cq_get_device_error -- synchronise `stream`, then read and clear the
+ * device error word of the current device.  Returns CQ_OK when no bounded
+ * wait ran out since the last call, CQ_ERR_TIMEOUT otherwise (the site code
+ * of the first wait that gave up is stored in *site when site != NULL).
+ */
+CQ_API int cq_get_device_error(void *stream, int *site);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CQ_H_ */
