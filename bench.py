@@ -1,0 +1,459 @@
+"""Benchmark of the CubicQuant weight-only GEMM on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+                    [--workload down_m1|gate_up_m1|...] [--no-secondary]
+
+Headline workload (default): the Kimi-K3-shaped expert down_proj stored as
+CubicQuant W3 G512, N = 7168 x K = 3072, one activation row (M = 1).  One
+step is one fused GEMM (unpack -> level generation -> tcgen05 MMA -> output)
+over one weight copy; consecutive steps rotate through R distinct copies
+whose total size exceeds 4x the L2 cache, so every step streams its packed
+weights from HBM.  Metric: packed-weight GB/s = N*K*(B + 64/G)/8 bytes per
+step / time per step (x and y excluded, as the metric defines it).
+
+Timing: W untimed warm-up steps, then exactly K steps captured in one CUDA
+graph and bracketed by CUDA events on the launching stream, with a barrier
+and device synchronisation on both sides; under torchrun each rank runs its
+own replica (no collective on the data path) and the slowest rank's time is
+used.  Rank 0 prints one JSON line.
+
+--impl reference runs the CPU oracle (FP64, plain C) on a bounded sample of
+the same workload instead, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "Cubic GEMM packed-weight GB/s at M=1 and TFLOP/s at M>=256, % of B200 roofline"
+
+WORKLOADS = {
+    # name: (description, N, K, B, G, M, epilogue)
+    "down_m1": ("Kimi-K3 expert down_proj, CubicQuant W3 G512, N=7168 x K=3072, M=1",
+                7168, 3072, 3, 512, 1, 0),
+    "gate_up_m1": ("Kimi-K3 expert gate+up, CubicQuant W2 G512, N=6144 x K=7168, M=1, SwiGLU",
+                   6144, 7168, 2, 512, 1, 1),
+    "down_m16": ("Kimi-K3 expert down_proj, W3 G512, N=7168 x K=3072, M=16",
+                 7168, 3072, 3, 512, 16, 0),
+    "gate_up_m4096": ("Kimi-K3 expert gate+up, W2 G512, N=6144 x K=7168, M=4096, SwiGLU",
+                      6144, 7168, 2, 512, 4096, 1),
+    "down_m4096": ("Kimi-K3 expert down_proj, W3 G512, N=7168 x K=3072, M=4096",
+                   7168, 3072, 3, 512, 4096, 0),
+}
+
+
+def packed_bytes(N, K, B, G):
+    return N * K * B // 8 + N * (K // G) * 8
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(
+            d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# --------------------------------------------------------------------------
+# clock sampling (NVML) during the timed region
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons = [], 0
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _poll(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                self.reasons |= n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self._sample_once()
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+        return self
+
+    def _sample_once(self):
+        try:
+            self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+            self.reasons |= self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            pass
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            self._sample_once()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": [k for k, v in self.REASONS.items() if self.reasons & v]}
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (replicas only; no data-path collective)
+# --------------------------------------------------------------------------
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------
+
+def build_weights(cq, name, device):
+    import synthetic
+    desc, N, K, B, G, M, epi = WORKLOADS[name]
+    codes, s, ab = synthetic.matrix(("bench", name), N, K, B, G, device=device)
+    packed = cq.cq_pack(codes, B)
+    del codes
+    return packed, s.contiguous(), ab.contiguous()
+
+
+def rotation_copies(nbytes, l2_bytes):
+    return max(2, int(np.ceil(4.5 * l2_bytes / nbytes)))
+
+
+def time_gemm(cq, name, steps, warmup, world, device, sample_clocks=False):
+    """Device-timed K steps of one workload (CUDA graph of K launches)."""
+    desc, N, K, B, G, M, epi = WORKLOADS[name]
+    import synthetic
+    packed, s, ab = build_weights(cq, name, device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    wbytes = packed_bytes(N, K, B, G)
+    R = rotation_copies(wbytes, l2) if M <= 64 else 1
+    copies = [(packed.clone(), s.clone(), ab.clone()) for _ in range(R)]
+    x = synthetic.activations(11, M, K).to(device)
+    ncol = N // 2 if epi else N
+    y = torch.empty((M, ncol), dtype=torch.float32, device=device)
+    ws = cq.gemm_workspace(M, N, K, B, G, epi, device)
+    stream = torch.cuda.Stream(device)
+
+    def step(i, st):
+        p, sc, a = copies[i % R]
+        cq.cq_gemm(x, p, sc, a, N, K, B, G, epilogue=epi, workspace=ws, out=y, stream=st)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(warmup, 3)):
+            step(i, stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            step(i, stream)
+    # one untimed replay (graph upload) before timing
+    g.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    with sampler if sample_clocks else _null():
+        ev0.record(stream)
+        with torch.cuda.stream(stream):
+            g.replay()
+        ev1.record(stream)
+        ev1.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms, world)
+    st, site = cq.device_error()
+    if st != 0:
+        raise RuntimeError(f"device wait timed out (site {site})")
+    del g
+    flops = 2.0 * M * N * K
+    res = dict(name=name, desc=desc, M=M, N=N, K=K, B=B, G=G, epilogue=epi, R=R,
+               rot_mb=R * wbytes / 1e6, ms_total=ms, ms_per_step=ms / steps,
+               wbytes=wbytes, gbs=wbytes * steps / (ms * 1e-3) / 1e9,
+               tflops=flops * steps / (ms * 1e-3) / 1e12,
+               alg_bytes=wbytes + M * K * 2 + M * ncol * 4,
+               clocks=sampler.summary() if sample_clocks else None)
+    return res
+
+
+class _null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def time_e2e(cq, name, steps, device):
+    """End to end through the public API: per step, pinned-host x -> device,
+    cq_gemm, y -> pinned host, with ordinary (non-graph) calls."""
+    desc, N, K, B, G, M, epi = WORKLOADS[name]
+    import synthetic
+    packed, s, ab = build_weights(cq, name, device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    wbytes = packed_bytes(N, K, B, G)
+    R = rotation_copies(wbytes, l2) if M <= 64 else 1
+    copies = [(packed.clone(), s.clone(), ab.clone()) for _ in range(R)]
+    xh = synthetic.activations(12, M, K).pin_memory()
+    ncol = N // 2 if epi else N
+    yh = torch.empty((M, ncol), dtype=torch.float32).pin_memory()
+    xd = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+    yd = torch.empty((M, ncol), dtype=torch.float32, device=device)
+    ws = cq.gemm_workspace(M, N, K, B, G, epi, device)
+    stream = torch.cuda.Stream(device)
+    n = max(10, min(steps, 2000))
+
+    def one(i):
+        p, sc, a = copies[i % R]
+        xd.copy_(xh, non_blocking=True)
+        cq.cq_gemm(xd, p, sc, a, N, K, B, G, epilogue=epi, workspace=ws, out=yd, stream=stream)
+        yh.copy_(yd, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(5):
+            one(i)
+        stream.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for i in range(n):
+            one(i)
+        ev1.record(stream)
+        ev1.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    return {"value": round(wbytes * n / (ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * ncol * 4,
+            "steps": n, "ms_per_step": ms / n}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline)
+# --------------------------------------------------------------------------
+
+def oracle_sample(name, rows):
+    import oracle
+    import synthetic
+    desc, N, K, B, G, M, epi = WORKLOADS[name]
+    codes, s, ab = synthetic.matrix(("bench", name), N, K, B, G, nrows=rows)
+    packed = oracle.pack(codes.numpy(), B)
+    x = synthetic.activations(11, M, K).view(torch.int16).numpy().view(np.uint16)
+    return (oracle, packed, s.numpy(), ab.view(torch.int16).numpy().view(np.uint16), x,
+            rows, K, B, G)
+
+
+def time_oracle(name, rows, min_seconds=0.0, reps=1):
+    oracle, packed, s, ab, x, rows, K, B, G = oracle_sample(name, rows)
+    wbytes = packed_bytes(rows, K, B, G)
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.gemm(x, packed, s, ab, rows, K, B, G)
+        n += 1
+        el = time.perf_counter() - t0
+        if n >= reps and el >= min_seconds:
+            break
+    return wbytes * n / el / 1e9, el, n, oracle.num_threads()
+
+
+def cpu_baseline(name):
+    desc, N, K, B, G, M, epi = WORKLOADS[name]
+    gbs, el, n, cores = time_oracle(name, N, min_seconds=10.0)
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"the full {N}x{K} W{B} G{G} matrix at M={M}, {n} pass(es), "
+                      f"{el:.1f} s, FP64 plain C over {cores} threads"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    name = args.workload
+    desc, N, K, B, G, M, epi = WORKLOADS[name]
+    rows = min(N, 1024)
+    oracle, packed, s, ab, x, rows, K, B, G = oracle_sample(name, rows)
+    wbytes = packed_bytes(rows, K, B, G)
+    for _ in range(max(args.warmup, 0)):
+        oracle.gemm(x, packed, s, ab, rows, K, B, G)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.gemm(x, packed, s, ab, rows, K, B, G)
+    el = time.perf_counter() - t0
+    val = wbytes * args.steps / el / 1e9
+    cores = oracle.num_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": desc, "M": M, "N": N, "K": K, "B": B, "G": G},
+        "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"{rows} of {N} weight rows per step at M={M}"},
+        "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--workload", default="down_m1", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        return run_reference(args, world, rank)
+
+    import bit_non_uniform_b200 as cq
+    world, rank, local = dist_setup(args)
+    device = torch.device("cuda", torch.cuda.current_device())
+    hbm, tf_burst, tf_sust, peak_src = load_peaks()
+
+    main_res = time_gemm(cq, args.workload, args.steps, args.warmup, world, device,
+                         sample_clocks=True)
+    secondary = []
+    if not args.no_secondary:
+        for name in ["gate_up_m1", "down_m16", "gate_up_m4096", "down_m4096"]:
+            if name == args.workload:
+                continue
+            steps = 400 if WORKLOADS[name][5] <= 64 else 20
+            r = time_gemm(cq, name, steps, 3, world, device)
+            bound = "hbm" if r["M"] <= 64 else "tensor"
+            ent = {"workload": r["desc"], "ms_per_step": round(r["ms_per_step"], 5),
+                   "packed_gbs": round(r["gbs"] * world, 1),
+                   "tflops": round(r["tflops"] * world, 2)}
+            if bound == "hbm":
+                ach = r["alg_bytes"] / (r["ms_per_step"] * 1e-3) / 1e9
+                ent["roofline"] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
+                                   "unit": "GB/s", "frac": round(ach / hbm, 4)}
+            else:
+                ent["roofline"] = {"bound": "tensor", "achieved": round(r["tflops"], 1),
+                                   "peak": tf_burst, "unit": "TFLOP/s",
+                                   "frac": round(r["tflops"] / tf_burst, 4)}
+            secondary.append(ent)
+
+    e2e = time_e2e(cq, args.workload, args.steps, device)
+    e2e["value"] = round(e2e["value"] * world, 3)
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
+
+    r = main_res
+    value = r["gbs"] * world          # every rank streams its own replica
+    ach = r["alg_bytes"] / (r["ms_per_step"] * 1e-3) / 1e9
+    traffic = None
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(r["ms_per_step"], 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": r["desc"], "M": r["M"], "N": r["N"], "K": r["K"],
+                   "B": r["B"], "G": r["G"], "bytes_per_step": r["wbytes"],
+                   "l2": f"inputs larger than L2: {r['R']} rotating weight copies, "
+                         f"{r['rot_mb']:.0f} MB",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(ach / hbm, 4), "traffic": traffic,
+                     "peak_source": peak_src},
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": r["clocks"],
+        "secondary": secondary,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

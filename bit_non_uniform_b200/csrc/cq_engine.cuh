@@ -8,20 +8,26 @@
 // sums the partial tiles in CTA order (deterministic) and applies the
 // epilogue.
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warps 0-3  decoders: thread i owns weight row i of the tile and TMEM
 //              lane i.  Per group it builds a private BF16 pair table
 //              (two codes -> two levels, one 32-bit word per entry, the
 //              entries of all 128 threads interleaved so that every lookup
 //              hits the thread's own bank), then turns each slice of packed
 //              codes into 64 BF16x2 words written to TMEM with tcgen05.st
-//              (the A operand of the MMA).  They also run the epilogue.
-//   warp 4     producer: 1-D bulk copies of the packed rows and 2-D TMA
-//              loads of the activation tile (128-byte swizzle) into a ring
-//              of shared-memory stages.
+//              (the A operand of the MMA).
+//   warp 4     producer: 2-D TMA loads into a ring of shared-memory
+//              stages: per 128-code slice, two boxes of 64 weight rows x
+//              16*B bytes of packed codes (32-byte swizzle for W2, 64-byte
+//              for W4, none for W3's 48-byte rows, so the decoders'
+//              row-per-thread 16-byte reads are bank-conflict free), and the
+//              activation tile as 64-column boxes with the 128-byte swizzle.
 //   warp 5     TMEM owner and MMA issuer: tcgen05.mma kind::f16 with A from
 //              TMEM (decoded weights) and B from shared memory
-//              (activations), FP32 accumulators in TMEM.
+//              (activations), FP32 accumulators in TMEM, double-buffered so
+//              the next tile's MMAs overlap the previous tile's epilogue.
+//   warps 6-9  epilogue: tcgen05.ld of the accumulator, output conversion,
+//              SwiGLU, stream-K partials and their reduction.
 //
 // This follows the article's fused A16 path ("压缩权重必须“边解码、边计算”"):
 // packed codes + group parameters -> unpack and generate the levels inside
@@ -38,30 +44,31 @@ namespace cq {
 
 constexpr int kRows = 128;            // weight rows per tile (MMA M)
 constexpr int kSlice = 128;           // codes per slice along K
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kTmemCols = 512;
 constexpr int kTmemRing = 4;          // TMEM slice buffers (64 columns each)
-constexpr int kDCol = 256;            // first TMEM column of the accumulator
+constexpr int kDCol = 256;            // first TMEM column of the accumulators
 constexpr int kDecoders = 128;
+constexpr int kEpilogue = 128;
+constexpr int kEpiWarp0 = 6;
 
 template <int NT>
 struct EngineCfg {
   static constexpr int SPS = NT <= 32 ? 4 : (NT == 64 ? 2 : 1);   // slices per stage
-  static constexpr int pitch(int B) {                           // smem row pitch, odd # of 16B
-    return ((SPS * B) % 2 ? SPS * B : SPS * B + 1) * 16;
-  }
-  static constexpr int W_BYTES = ((kRows * pitch(4) + 1023) / 1024) * 1024;
+  static constexpr int SLICE_W_BYTES = kRows * 16 * 4;          // one slice of packed rows (B<=4)
+  static constexpr int W_BYTES = SPS * SLICE_W_BYTES;
   static constexpr int X_BYTES = 256 * SPS * NT;                // 2*SPS boxes of 64 x NT bf16
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
-  static constexpr int TBL_BYTES = 64 * 512;                    // largest pair table (W3)
   static constexpr int XCHG_BYTES = 16 * 64 * 4;
   static constexpr int MISC_BYTES = 1024;
-  static constexpr int BUDGET = 224 * 1024;
-  static constexpr int S_RAW = (BUDGET - 1024 - TBL_BYTES - XCHG_BYTES - MISC_BYTES) / STAGE_BYTES;
+  static constexpr int TBL_BYTES = 64 * 512;                    // static pair table (W3 size)
+  static constexpr int BUDGET = 226 * 1024 - TBL_BYTES;         // dynamic part
+  static constexpr int S_RAW = (BUDGET - 1024 - XCHG_BYTES - MISC_BYTES) / STAGE_BYTES;
   static constexpr int S = S_RAW > 6 ? 6 : S_RAW;
-  static constexpr int SMEM = 1024 + S * STAGE_BYTES + TBL_BYTES + XCHG_BYTES + MISC_BYTES;
+  static constexpr int SMEM = 1024 + S * STAGE_BYTES + XCHG_BYTES + MISC_BYTES;
   static_assert(S >= 2, "not enough shared memory for two stages");
-  static_assert(SMEM <= 227 * 1024, "shared memory budget exceeded");
+  static_assert(SMEM + TBL_BYTES <= 227 * 1024, "shared memory budget exceeded");
+  static_assert(kDCol + 2 * NT <= kTmemCols, "TMEM budget exceeded");
 };
 
 // One quantized matrix operand.
@@ -96,7 +103,26 @@ struct EngineParams {
   // control
   uint64_t timeout_ns;
   int debug_skip_first_stage;   // test hook: never issue stage load 0
+  uint64_t* trace;              // optional [P][64] profile counters, or null
 };
+
+// Optional per-role cycle accounting into p.trace: PROF_MARK starts an
+// interval, PROF_ADD(k) adds the cycles since the mark to counter k,
+// PROF_FLUSH(base) stores the 8 counters at slots base..base+7 of this CTA.
+#define PROF_MARK() (prof_t = p.trace ? clock64() : 0)
+#define PROF_ADD(k)                                                         \
+  do {                                                                      \
+    if (p.trace) {                                                          \
+      const long long now_ = clock64();                                     \
+      prof[(k)] += now_ - prof_t;                                           \
+      prof_t = now_;                                                        \
+    }                                                                       \
+  } while (0)
+#define PROF_FLUSH(base)                                                    \
+  do {                                                                      \
+    if (p.trace)                                                            \
+      for (int k_ = 0; k_ < 8; ++k_) p.trace[blockIdx.x * 64 + (base) + k_] = prof[k_]; \
+  } while (0)
 
 struct TileInfo {
   MatrixRef mat;
@@ -132,102 +158,152 @@ __device__ __forceinline__ int owner_of(int64_t W, int P, int64_t x) {
   return static_cast<int>(((x + 1) * P - 1) / W);
 }
 
+// One segment of a CTA's range: the slices [s0, s1) of tile t.
+struct Segment {
+  int t, s0, s1;
+  int64_t end;
+};
+__device__ __forceinline__ Segment segment_at(int64_t x, int64_t r1, int spt) {
+  Segment g;
+  g.t = static_cast<int>(x / spt);
+  const int64_t tbeg = static_cast<int64_t>(g.t) * spt;
+  g.s0 = static_cast<int>(x - tbeg);
+  g.end = tbeg + spt < r1 ? tbeg + spt : r1;
+  g.s1 = static_cast<int>(g.end - tbeg);
+  return g;
+}
+
+// Wait with an inline fast path; the bounded slow path is out of line.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort,
+                                           uint64_t timeout_ns, int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait(bar, parity, abort, timeout_ns, site);
+}
+
 // ---------------------------------------------------------------------------
 // decoder helpers
 // ---------------------------------------------------------------------------
 
-// Build this thread's pair table for one group: 2^B levels
-// L_u = BF16(FP32(s sign q(t_u))) and the entries
+// Pair-table layout in shared memory: entry e of tile row i is the 32-bit
+// word at tbl + e*512 + 4*i, so the lookups of a warp always hit 32
+// distinct banks.  Entries:
 //   B=2: e = u0 | u1<<2 (16 entries)  ->  L[u0] | L[u1] << 16
 //   B=3: e = u0 | u1<<3 (64 entries)  ->  L[u0] | L[u1] << 16
 //   B=4: e = u        (16 entries)   ->  L[u]  | L[u]  << 16
-// Entry e of thread i lives at tbl + e*512 + 4*i.
+// with L_u = BF16(FP32(s sign(k) q(t))) the level of code u.  Levels are odd
+// in k (q(t) carries the sign), so only the positive side is evaluated in
+// FP64 and the negative codes flip the BF16 sign bit.
 template <int B>
-__device__ __forceinline__ void build_table(uint32_t tbase, bool valid, float s, uint32_t abw,
-                                            int mode) {
+__device__ __forceinline__ void build_table(uint32_t tbl, uint32_t tid4, bool valid, float s,
+                                            uint32_t abw, int mode) {
+  constexpr int H = 1 << (B - 1);
   uint32_t L[1 << B];
   if (valid) {
     const double a = static_cast<double>(__half2float(__ushort_as_half(abw & 0xFFFFu)));
     const double b = static_cast<double>(__half2float(__ushort_as_half(abw >> 16)));
+    if (mode == CQ_GRID_MIDRISE) {
+      // codes H+j (j = 0..H-1) are the positive side, H-1-j their mirror
 #pragma unroll
-    for (int u = 0; u < (1 << B); ++u)
-      L[u] = bf16_bits(static_cast<float>(level_f64(u, B, mode, s, a, b)));
+      for (int j = 0; j < H; ++j) {
+        const uint32_t m = bf16_bits(static_cast<float>(level_f64(H + j, B, 0, s, a, b)));
+        L[H + j] = m;
+        L[H - 1 - j] = m ^ 0x8000u;
+      }
+    } else {
+      // Kc = H-1; code Kc+m has |k| = m (m = 0..H), code Kc-m its mirror
+#pragma unroll
+      for (int m = 0; m <= H; ++m) {
+        const uint32_t v = bf16_bits(static_cast<float>(level_f64(H - 1 + m, B, 1, s, a, b)));
+        L[H - 1 + m] = v;
+        if (m >= 1 && m <= H - 1) L[H - 1 - m] = v ^ 0x8000u;
+      }
+    }
   } else {
 #pragma unroll
     for (int u = 0; u < (1 << B); ++u) L[u] = 0u;
   }
   if constexpr (B == 2) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) sts32(tbase + e * 512, L[e & 3] | (L[e >> 2] << 16));
+    for (int e = 0; e < 16; ++e) sts32(tbl + (e << 9) + tid4, L[e & 3] | (L[e >> 2] << 16));
   } else if constexpr (B == 3) {
 #pragma unroll
-    for (int e = 0; e < 64; ++e) sts32(tbase + e * 512, L[e & 7] | (L[e >> 3] << 16));
+    for (int e = 0; e < 64; ++e) sts32(tbl + (e << 9) + tid4, L[e & 7] | (L[e >> 3] << 16));
   } else {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) sts32(tbase + e * 512, L[e] | (L[e] << 16));
+    for (int e = 0; e < 16; ++e) sts32(tbl + (e << 9) + tid4, L[e] | (L[e] << 16));
   }
+}
+
+// Bits [sh, sh+6) of word w moved to bit 9 (the table's entry stride).
+__device__ __forceinline__ uint32_t at_bit9(uint32_t w, int sh) {
+  return sh >= 9 ? (w >> (sh - 9)) : (w << (9 - sh));
 }
 
 // Decode pairs [P0, P0+32) of one 128-code slice (codes in c[]) into r[].
 template <int B, int P0>
-__device__ __forceinline__ void decode_half(const uint32_t (&c)[4 * B], uint32_t tbase,
-                                            uint32_t (&r)[32]) {
+__device__ __forceinline__ void decode_half(const uint32_t (&c)[4 * B], uint32_t tbl,
+                                            uint32_t tid4, uint32_t (&r)[32]) {
 #pragma unroll
   for (int q = 0; q < 32; ++q) {
     const int p = P0 + q;
     if constexpr (B == 2) {
-      const uint32_t idx = (c[p >> 3] >> (4 * (p & 7))) & 15u;
-      r[q] = lds32(tbase + (idx << 9));
+      const uint32_t v = at_bit9(c[p >> 3], 4 * (p & 7));
+      r[q] = lds32(tbl + ((v & (15u << 9)) | tid4));
     } else if constexpr (B == 3) {
       const int o = 6 * p;
       const int wi = o >> 5, sh = o & 31;
       uint32_t v;
       if (sh <= 26)
-        v = c[wi] >> sh;
+        v = at_bit9(c[wi], sh);
       else
-        v = __funnelshift_r(c[wi], c[wi + 1 < 4 * B ? wi + 1 : 4 * B - 1], sh);
-      r[q] = lds32(tbase + ((v & 63u) << 9));
+        v = __funnelshift_r(c[wi], c[wi + 1 < 4 * B ? wi + 1 : 4 * B - 1], sh - 9);
+      r[q] = lds32(tbl + ((v & (63u << 9)) | tid4));
     } else {
-      const uint32_t byte = (c[p >> 2] >> (8 * (p & 3))) & 0xFFu;
-      const uint32_t lo = lds32(tbase + ((byte & 15u) << 9));
-      const uint32_t hi = lds32(tbase + ((byte >> 4) << 9));
+      const int sh = 8 * (p & 3);
+      const uint32_t w = c[p >> 2];
+      const uint32_t lo = lds32(tbl + ((at_bit9(w, sh) & (15u << 9)) | tid4));
+      const uint32_t hi = lds32(tbl + ((at_bit9(w, sh + 4) & (15u << 9)) | tid4));
       r[q] = __byte_perm(lo, hi, 0x7610);
     }
   }
 }
 
 template <int B>
-__device__ __forceinline__ void decode_slice_to_tmem(uint32_t codes_addr, uint32_t tbase,
+__device__ __forceinline__ void decode_slice_to_tmem(uint32_t codes_addr, uint32_t swz,
+                                                     uint32_t tbl, uint32_t tid4,
                                                      uint32_t taddr) {
   uint32_t c[4 * B];
 #pragma unroll
   for (int v = 0; v < B; ++v) {
-    const uint4 q = lds128(codes_addr + 16 * v);
+    const uint4 q = lds128(codes_addr + 16 * (v ^ swz));
     c[4 * v + 0] = q.x;
     c[4 * v + 1] = q.y;
     c[4 * v + 2] = q.z;
     c[4 * v + 3] = q.w;
   }
   uint32_t r[32];
-  decode_half<B, 0>(c, tbase, r);
+  decode_half<B, 0>(c, tbl, tid4, r);
   tmem_st32(taddr, r);
-  decode_half<B, 32>(c, tbase, r);
+  decode_half<B, 32>(c, tbl, tid4, r);
   tmem_st32(taddr + 32, r);
 }
 
-__device__ __forceinline__ void named_bar_decoders() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+// ---------------------------------------------------------------------------
+// epilogue helpers (warps 6-9, named barrier 2)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void named_bar_epilogue() {
+  asm volatile("bar.sync 2, 128;" ::: "memory");
 }
 
-// All-decoders AND-vote at named barrier 1.  Every decoder reaches it once
-// per segment, whether or not one of its waits gave up, so the named
-// barriers of the epilogue are only entered when all 128 agree.
-__device__ __forceinline__ bool vote_all_decoders(bool ok) {
+// All-epilogue-threads AND-vote at named barrier 2.  Every epilogue thread
+// reaches it once per segment, whether or not one of its waits gave up, so
+// the epilogue's named barriers are only entered when all 128 agree.
+__device__ __forceinline__ bool vote_all_epilogue(bool ok) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "bar.red.and.pred q, 2, 128, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
       : "r"(static_cast<uint32_t>(ok))
@@ -237,7 +313,7 @@ __device__ __forceinline__ bool vote_all_decoders(bool ok) {
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
-// Store 16 accumulator columns (tokens m0..m0+15) of tile row i.
+// Store 16 accumulator columns (tokens m0..m0+15 of the tile) of tile row i.
 __device__ __forceinline__ void finalize16(const EngineParams& p, const TileInfo& ti, int i,
                                            int grow, const float (&v)[16], int cc,
                                            float* xchg) {
@@ -247,7 +323,7 @@ __device__ __forceinline__ void finalize16(const EngineParams& p, const TileInfo
 #pragma unroll
       for (int q = 0; q < 16; ++q) xchg[q * 64 + (i - 64)] = v[q];
     }
-    named_bar_decoders();
+    named_bar_epilogue();
     if (i < 64) {
       const int col = ti.rt * 64 + i;
 #pragma unroll
@@ -263,7 +339,7 @@ __device__ __forceinline__ void finalize16(const EngineParams& p, const TileInfo
         }
       }
     }
-    named_bar_decoders();
+    named_bar_epilogue();
   } else {
     if (grow < p.N) {
 #pragma unroll
@@ -287,26 +363,28 @@ __device__ __forceinline__ void finalize16(const EngineParams& p, const TileInfo
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     engine_kernel(const __grid_constant__ EngineParams p,
-                  const __grid_constant__ CUtensorMap xmap) {
+                  const __grid_constant__ CUtensorMap xmap,
+                  const __grid_constant__ CUtensorMap wmap) {
   using C = EngineCfg<NT>;
+  __shared__ __align__(32768) uint32_t s_tbl[64 * kRows];   // per-row pair tables
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-align the working area (swizzled TMA destinations need it)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   const uint32_t stage0 = base;
-  const uint32_t tbl = stage0 + C::S * C::STAGE_BYTES;
-  const uint32_t xchg_s = tbl + C::TBL_BYTES;
+  const uint32_t xchg_s = stage0 + C::S * C::STAGE_BYTES;
   const uint32_t misc = xchg_s + C::XCHG_BYTES;
   uint8_t* const gbase = smem_raw + (base - raw);
   float* const xchg = reinterpret_cast<float*>(gbase + (xchg_s - base));
+  const uint32_t tbl = smem_u32(s_tbl);
   // barriers and flags
   const uint32_t bar_full = misc;                         // [S]
   const uint32_t bar_wempty = bar_full + 8 * C::S;        // [S]
   const uint32_t bar_aready = bar_wempty + 8 * C::S;      // [4]
   const uint32_t bar_tfree = bar_aready + 8 * kTmemRing;  // [4]
-  const uint32_t bar_dfull = bar_tfree + 8 * kTmemRing;
-  const uint32_t bar_dfree = bar_dfull + 8;
-  const uint32_t bar_fin = bar_dfree + 8;
+  const uint32_t bar_dfull = bar_tfree + 8 * kTmemRing;   // [2]
+  const uint32_t bar_dfree = bar_dfull + 16;              // [2]
+  const uint32_t bar_fin = bar_dfree + 16;
   const uint32_t slot_tmem = bar_fin + 8;
   volatile int* const abort_flag =
       reinterpret_cast<volatile int*>(gbase + (slot_tmem + 8 - base));
@@ -317,6 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int cta = blockIdx.x;
+  const long long prof_start = clock64();
+  long long prof[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  long long prof_t = 0;
 
   if (tid == 0) {
     for (int s = 0; s < C::S; ++s) {
@@ -327,8 +408,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_aready + 8 * s, kDecoders);
       mbar_init(bar_tfree + 8 * s, 1);
     }
-    mbar_init(bar_dfull, 1);
-    mbar_init(bar_dfree, kDecoders);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_dfull + 8 * s, 1);
+      mbar_init(bar_dfree + 8 * s, kEpilogue);
+    }
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
     *last_flag = 0;
@@ -339,7 +422,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
     tc_fence_before();
   }
-  if (warp == 4 && lane == 0) prefetch_tensormap(&xmap);
+  if (warp == 4 && lane == 0) {
+    prefetch_tensormap(&xmap);
+    prefetch_tensormap(&wmap);
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base =
@@ -355,62 +441,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     int st = 0;
     uint32_t round = 0;
     int load_no = 0;
-    int64_t x = r0;
-    while (x < r1 && !*abort_flag) {
-      const int t = static_cast<int>(x / p.spt);
-      const int s0 = static_cast<int>(x - static_cast<int64_t>(t) * p.spt);
-      const int64_t seg_end = static_cast<int64_t>(t + 1) * p.spt < r1
-                                  ? static_cast<int64_t>(t + 1) * p.spt
-                                  : r1;
-      const int s1 = static_cast<int>(seg_end - static_cast<int64_t>(t) * p.spt);
-      const TileInfo ti = resolve_tile(p, t, NT);
+    for (int64_t x = r0; x < r1 && !*abort_flag;) {
+      const Segment sg = segment_at(x, r1, p.spt);
+      const TileInfo ti = resolve_tile(p, sg.t, NT);
       const int Bw = ti.mat.B;
-      const int pitch = C::pitch(Bw);
-      const int64_t row_bytes = static_cast<int64_t>(p.K) * Bw / 8;
-      int valid_rows = 0;
-      if (p.epilogue == CQ_EPI_SWIGLU) {
-        valid_rows = kRows;
-      } else {
-        const int rem = p.N - ti.rt * kRows;
-        valid_rows = rem < kRows ? rem : kRows;
-      }
-      for (int sb = s0; sb < s1; sb += C::SPS) {
-        const int ns = (s1 - sb) < C::SPS ? (s1 - sb) : C::SPS;
-        if (!mbar_wait(bar_wempty + 8 * st, (round & 1u) ^ 1u, abort_flag, tmo,
-                       SITE_PRODUCER_EMPTY))
+      // first weight row of the two 64-row boxes of this tile
+      const int row_a = tile_row(p, ti.rt, 0);
+      const int row_b = tile_row(p, ti.rt, 64);
+      for (int sb = sg.s0; sb < sg.s1; sb += C::SPS) {
+        const int ns = (sg.s1 - sb) < C::SPS ? (sg.s1 - sb) : C::SPS;
+        PROF_MARK();
+        if (!wait_phase(bar_wempty + 8 * st, (round & 1u) ^ 1u, abort_flag, tmo,
+                        SITE_PRODUCER_EMPTY))
           break;
+        PROF_ADD(0);
         const bool skip = p.debug_skip_first_stage && load_no == 0;
-        if (!skip) {
-          const uint32_t wb = static_cast<uint32_t>(ns * 16 * Bw);
-          const uint32_t bytes =
-              static_cast<uint32_t>(valid_rows) * wb + static_cast<uint32_t>(2 * ns * NT * 128);
+        if (!skip && lane == 0) {
+          const uint32_t wbox = 64u * 16u * Bw;                   // bytes of one weight box
+          const uint32_t bytes = static_cast<uint32_t>(ns) * (2u * wbox) +
+                                 static_cast<uint32_t>(2 * ns * NT * 128);
           const uint32_t wdst = stage0 + st * C::STAGE_BYTES;
           const uint32_t xdst = wdst + C::W_BYTES;
-          if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * st, bytes);
-          __syncwarp();
-          for (int r = lane; r < valid_rows; r += 32) {
-            const int grow = tile_row(p, ti.rt, r);
-            const uint8_t* src = ti.mat.packed + static_cast<int64_t>(grow) * row_bytes +
-                                 static_cast<int64_t>(sb) * 16 * Bw;
-            bulk_g2s(wdst + r * pitch, src, wb, bar_full + 8 * st);
+          mbar_arrive_expect_tx(bar_full + 8 * st, bytes);
+          for (int j = 0; j < ns; ++j) {
+            const int cb = (sb + j) * 16 * Bw;                   // byte column of the slice
+            const uint32_t sdst = wdst + j * C::SLICE_W_BYTES;
+            tma_load_2d(sdst, &wmap, cb, row_a, bar_full + 8 * st);
+            tma_load_2d(sdst + wbox, &wmap, cb, row_b, bar_full + 8 * st);
           }
-          if (lane == 0) {
-            for (int b = 0; b < 2 * ns; ++b)
-              tma_load_2d(xdst + b * (NT * 128), &xmap, sb * kSlice + b * 64, ti.x_row0,
-                          bar_full + 8 * st);
-          }
+          for (int b = 0; b < 2 * ns; ++b)
+            tma_load_2d(xdst + b * (NT * 128), &xmap, sb * kSlice + b * 64, ti.x_row0,
+                        bar_full + 8 * st);
         }
+        __syncwarp();
+        PROF_ADD(1);
+        prof[2] += 1;
         ++load_no;
         if (++st == C::S) {
           st = 0;
           ++round;
         }
       }
-      x = seg_end;
+      x = sg.end;
     }
-    // make sure no copy is still landing in shared memory before exit
+    if (lane == 0) PROF_FLUSH(8);
     __syncwarp();
     if (lane == 0 && *abort_flag) {
+      // make sure no copy is still landing in shared memory before exit:
       // the ring positions armed last are the only ones that may be in flight
       const int armed = load_no < C::S ? load_no : C::S;
       for (int k = 1; k <= armed; ++k) {
@@ -428,44 +505,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = idesc_bf16_f32(kRows, NT);
       int st = 0, ts = 0;
       uint32_t round = 0, tround = 0, seg = 0;
-      int64_t x = r0;
       bool ok = true;
-      while (ok && x < r1) {
-        const int t = static_cast<int>(x / p.spt);
-        const int s0 = static_cast<int>(x - static_cast<int64_t>(t) * p.spt);
-        const int64_t seg_end = static_cast<int64_t>(t + 1) * p.spt < r1
-                                    ? static_cast<int64_t>(t + 1) * p.spt
-                                    : r1;
-        const int s1 = static_cast<int>(seg_end - static_cast<int64_t>(t) * p.spt);
-        if (!mbar_wait(bar_dfree, (seg & 1u) ^ 1u, abort_flag, tmo, SITE_MMA_DFREE)) {
+      for (int64_t x = r0; ok && x < r1;) {
+        const Segment sg = segment_at(x, r1, p.spt);
+        const uint32_t db = seg & 1u;
+        PROF_MARK();
+        if (!wait_phase(bar_dfree + 8 * db, ((seg >> 1) & 1u) ^ 1u, abort_flag, tmo,
+                        SITE_MMA_DFREE)) {
           ok = false;
           break;
         }
+        PROF_ADD(0);
         tc_fence_after();
+        const uint32_t d_tmem = tmem_base + kDCol + db * NT;
         uint32_t acc = 0;
-        for (int sb = s0; sb < s1 && ok; sb += C::SPS) {
-          const int ns = (s1 - sb) < C::SPS ? (s1 - sb) : C::SPS;
-          if (!mbar_wait(bar_full + 8 * st, round & 1u, abort_flag, tmo, SITE_MMA_FULL)) {
+        for (int sb = sg.s0; sb < sg.s1 && ok; sb += C::SPS) {
+          const int ns = (sg.s1 - sb) < C::SPS ? (sg.s1 - sb) : C::SPS;
+          PROF_MARK();
+          if (!wait_phase(bar_full + 8 * st, round & 1u, abort_flag, tmo, SITE_MMA_FULL)) {
             ok = false;
             break;
           }
+          PROF_ADD(1);
           tc_fence_after();
-          const uint32_t xs = stage0 + st * C::STAGE_BYTES + C::W_BYTES;
+          const uint64_t desc0 = smem_desc_sw128(stage0 + st * C::STAGE_BYTES + C::W_BYTES);
           for (int j = 0; j < ns; ++j) {
-            if (!mbar_wait(bar_aready + 8 * ts, tround & 1u, abort_flag, tmo, SITE_MMA_AREADY)) {
+            PROF_MARK();
+            if (!wait_phase(bar_aready + 8 * ts, tround & 1u, abort_flag, tmo,
+                            SITE_MMA_AREADY)) {
               ok = false;
               break;
             }
+            PROF_ADD(2);
             tc_fence_after();
+            const uint32_t a0 = tmem_base + ts * 64;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-              const int kin = j * kSlice + kk * 16;           // k offset inside the stage
-              const uint32_t baddr = xs + (kin >> 6) * (NT * 128) + (kin & 63) * 2;
-              mma_ts_bf16(tmem_base + kDCol, tmem_base + ts * 64 + kk * 8,
-                          smem_desc_sw128(baddr), idesc, acc);
+              // activation box 2j + kk/4, 32-byte K step inside its 128-byte rows
+              const uint64_t off =
+                  static_cast<uint64_t>(((2 * j + (kk >> 2)) * NT * 128 + (kk & 3) * 32) >> 4);
+              mma_ts_bf16(d_tmem, a0 + kk * 8, desc0 + off, idesc, acc);
               acc = 1;
             }
             mma_commit(bar_tfree + 8 * ts);
+            PROF_ADD(3);
+            prof[4] += 1;
             if (++ts == kTmemRing) {
               ts = 0;
               ++tround;
@@ -479,54 +563,52 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        mma_commit(bar_dfull);
+        mma_commit(bar_dfull + 8 * db);
         ++seg;
-        x = seg_end;
+        x = sg.end;
       }
+      PROF_FLUSH(16);
       // all issued MMAs have completed before TMEM is released
       mma_commit(bar_fin);
       volatile int dummy = 0;
       mbar_wait(bar_fin, 0, &dummy, tmo, SITE_TEARDOWN);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 4) {
     // ------------------------------------------------------------ decoders
     const int i = tid;                                   // tile row / TMEM lane
-    const uint32_t tbase = tbl + 4u * i;
+    const uint32_t tid4 = 4u * i;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     int st = 0, ts = 0;
-    uint32_t round = 0, tround = 0, seg = 0;
-    int64_t x = r0;
+    uint32_t round = 0, tround = 0;
     bool ok = true;
     const int ng = p.K / p.G;
-    while (ok && x < r1) {
-      const int t = static_cast<int>(x / p.spt);
-      const int s0 = static_cast<int>(x - static_cast<int64_t>(t) * p.spt);
-      const int64_t seg_end = static_cast<int64_t>(t + 1) * p.spt < r1
-                                  ? static_cast<int64_t>(t + 1) * p.spt
-                                  : r1;
-      const int s1 = static_cast<int>(seg_end - static_cast<int64_t>(t) * p.spt);
-      const TileInfo ti = resolve_tile(p, t, NT);
+    for (int64_t x = r0; ok && x < r1;) {
+      const Segment sg = segment_at(x, r1, p.spt);
+      const TileInfo ti = resolve_tile(p, sg.t, NT);
       const int Bw = ti.mat.B;
-      const int pitch = C::pitch(Bw);
       const int grow = tile_row(p, ti.rt, i);
+      // 16-byte chunk v of this row sits at chunk (v ^ swz) of the row (TMA swizzle)
+      const uint32_t swz = Bw == 2 ? ((i >> 2) & 1u) : (Bw == 4 ? ((i >> 1) & 3u) : 0u);
       const bool valid = grow < p.N;
       // group metadata: the current group and a prefetch of the next one
       int cur_g = -1;
-      int g_next = (s0 * kSlice) / p.G;
+      int g_next = (sg.s0 * kSlice) / p.G;
       float s_next = 0.f;
       uint32_t ab_next = 0;
       if (valid) {
         s_next = __ldg(ti.mat.scales + static_cast<int64_t>(grow) * ng + g_next);
         ab_next = __ldg(ti.mat.ab + static_cast<int64_t>(grow) * ng + g_next);
       }
-      for (int sb = s0; sb < s1 && ok; sb += C::SPS) {
-        const int ns = (s1 - sb) < C::SPS ? (s1 - sb) : C::SPS;
-        if (!mbar_wait(bar_full + 8 * st, round & 1u, abort_flag, tmo, SITE_DECODER_FULL)) {
+      for (int sb = sg.s0; sb < sg.s1 && ok; sb += C::SPS) {
+        const int ns = (sg.s1 - sb) < C::SPS ? (sg.s1 - sb) : C::SPS;
+        PROF_MARK();
+        if (!wait_phase(bar_full + 8 * st, round & 1u, abort_flag, tmo, SITE_DECODER_FULL)) {
           ok = false;
           break;
         }
-        const uint32_t wrow = stage0 + st * C::STAGE_BYTES + i * pitch;
+        PROF_ADD(0);
+        const uint32_t wrow = stage0 + st * C::STAGE_BYTES + i * 16 * Bw;
         for (int j = 0; j < ns; ++j) {
           const int g = ((sb + j) * kSlice) / p.G;
           if (g != cur_g) {
@@ -540,29 +622,35 @@ __global__ void __launch_bounds__(kThreads, 1)
               ab_next = __ldg(ti.mat.ab + static_cast<int64_t>(grow) * ng + g_next);
             }
             if (Bw == 2)
-              build_table<2>(tbase, valid, s_cur, ab_cur, p.mode);
+              build_table<2>(tbl, tid4, valid, s_cur, ab_cur, p.mode);
             else if (Bw == 3)
-              build_table<3>(tbase, valid, s_cur, ab_cur, p.mode);
+              build_table<3>(tbl, tid4, valid, s_cur, ab_cur, p.mode);
             else
-              build_table<4>(tbase, valid, s_cur, ab_cur, p.mode);
+              build_table<4>(tbl, tid4, valid, s_cur, ab_cur, p.mode);
+            prof[7] += 1;
           }
-          if (!mbar_wait(bar_tfree + 8 * ts, (tround & 1u) ^ 1u, abort_flag, tmo,
-                         SITE_DECODER_TFREE)) {
+          PROF_ADD(1);
+          if (!wait_phase(bar_tfree + 8 * ts, (tround & 1u) ^ 1u, abort_flag, tmo,
+                          SITE_DECODER_TFREE)) {
             ok = false;
             break;
           }
+          PROF_ADD(2);
           tc_fence_after();
           const uint32_t taddr = tmem_base + lane_off + ts * 64;
-          const uint32_t caddr = wrow + j * 16 * Bw;
+          const uint32_t caddr = wrow + j * C::SLICE_W_BYTES;
           if (Bw == 2)
-            decode_slice_to_tmem<2>(caddr, tbase, taddr);
+            decode_slice_to_tmem<2>(caddr, swz, tbl, tid4, taddr);
           else if (Bw == 3)
-            decode_slice_to_tmem<3>(caddr, tbase, taddr);
+            decode_slice_to_tmem<3>(caddr, swz, tbl, tid4, taddr);
           else
-            decode_slice_to_tmem<4>(caddr, tbase, taddr);
+            decode_slice_to_tmem<4>(caddr, swz, tbl, tid4, taddr);
+          PROF_ADD(3);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(bar_aready + 8 * ts);
+          PROF_ADD(4);
+          prof[6] += 1;
           if (++ts == kTmemRing) {
             ts = 0;
             ++tround;
@@ -575,17 +663,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++round;
         }
       }
-      // ---------------------------------------------------------- epilogue
-      if (ok && !mbar_wait(bar_dfull, seg & 1u, abort_flag, tmo, SITE_DECODER_DFULL))
+      x = sg.end;
+    }
+    if (i == 0) PROF_FLUSH(24);
+    if (i == 127) PROF_FLUSH(32);
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                              // TMEM lane quarter
+    const int i = q * 32 + lane;                         // tile row
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    uint32_t seg = 0;
+    bool ok = true;
+    for (int64_t x = r0; ok && x < r1;) {
+      const Segment sg = segment_at(x, r1, p.spt);
+      const TileInfo ti = resolve_tile(p, sg.t, NT);
+      const int grow = tile_row(p, ti.rt, i);
+      const uint32_t db = seg & 1u;
+      PROF_MARK();
+      if (!wait_phase(bar_dfull + 8 * db, (seg >> 1) & 1u, abort_flag, tmo, SITE_DECODER_DFULL))
         ok = false;
-      if (!vote_all_decoders(ok)) {
+      if (!vote_all_epilogue(ok)) {
         ok = false;
         break;
       }
+      PROF_ADD(0);
       tc_fence_after();
-      const uint32_t daddr = tmem_base + lane_off + kDCol;
+      const uint32_t daddr = tmem_base + lane_off + kDCol + db * NT;
       const int nchunks = (ti.m_valid + 15) >> 4;
-      if (s0 == 0 && s1 == p.spt) {
+      if (sg.s0 == 0 && sg.s1 == p.spt) {
         // whole tile in this CTA: straight to the output
         for (int cc = 0; cc < nchunks; ++cc) {
           uint32_t rr[16];
@@ -593,63 +698,66 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           float v[16];
 #pragma unroll
-          for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(rr[q]);
+          for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(rr[k]);
           finalize16(p, ti, i, grow, v, cc, xchg);
         }
         tc_fence_before();
-        mbar_arrive(bar_dfree);
+        mbar_arrive(bar_dfree + 8 * db);
       } else {
         // partial tile: park it in the workspace, the last contributor reduces
         const int first_tile = static_cast<int>(r0 / p.spt);
-        const int slot = 2 * cta + (t == first_tile ? 0 : 1);
+        const int slot = 2 * cta + (sg.t == first_tile ? 0 : 1);
         float* const mine = p.partial + static_cast<int64_t>(slot) * NT * kRows;
         for (int cc = 0; cc < nchunks; ++cc) {
           uint32_t rr[16];
           tmem_ld16(daddr + cc * 16, rr);
           tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 16; ++q)
-            if (cc * 16 + q < ti.m_valid) mine[(cc * 16 + q) * kRows + i] = __uint_as_float(rr[q]);
+          for (int k = 0; k < 16; ++k)
+            if (cc * 16 + k < ti.m_valid) mine[(cc * 16 + k) * kRows + i] = __uint_as_float(rr[k]);
         }
         tc_fence_before();
-        mbar_arrive(bar_dfree);
+        mbar_arrive(bar_dfree + 8 * db);
         __threadfence();
-        named_bar_decoders();
-        const int64_t W_ = W;
-        const int c_lo = owner_of(W_, p.P, static_cast<int64_t>(t) * p.spt);
-        const int c_hi = owner_of(W_, p.P, static_cast<int64_t>(t) * p.spt + p.spt - 1);
+        named_bar_epilogue();
+        const int c_lo = owner_of(W, p.P, static_cast<int64_t>(sg.t) * p.spt);
+        const int c_hi = owner_of(W, p.P, static_cast<int64_t>(sg.t) * p.spt + p.spt - 1);
         if (i == 0) {
-          const int old = atomicAdd(p.counter + t, 1);
+          const int old = atomicAdd(p.counter + sg.t, 1);
           *last_flag = (old == c_hi - c_lo) ? 1 : 0;
         }
-        named_bar_decoders();
+        named_bar_epilogue();
         const bool last = *last_flag != 0;
         if (last) {
           __threadfence();
           for (int cc = 0; cc < nchunks; ++cc) {
             float v[16];
 #pragma unroll
-            for (int q = 0; q < 16; ++q) v[q] = 0.f;
+            for (int k = 0; k < 16; ++k) v[k] = 0.f;
             for (int c = c_lo; c <= c_hi; ++c) {
-              const int ft = static_cast<int>(range_begin(W_, p.P, c) / p.spt);
-              const int sl = 2 * c + (t == ft ? 0 : 1);
+              const int ft = static_cast<int>(range_begin(W, p.P, c) / p.spt);
+              const int sl = 2 * c + (sg.t == ft ? 0 : 1);
               const float* src = p.partial + static_cast<int64_t>(sl) * NT * kRows;
 #pragma unroll
-              for (int q = 0; q < 16; ++q)
-                if (cc * 16 + q < ti.m_valid) v[q] += __ldcg(src + (cc * 16 + q) * kRows + i);
+              for (int k = 0; k < 16; ++k)
+                if (cc * 16 + k < ti.m_valid) v[k] += __ldcg(src + (cc * 16 + k) * kRows + i);
             }
             finalize16(p, ti, i, grow, v, cc, xchg);
           }
-          if (i == 0) p.counter[t] = 0;
+          if (i == 0) p.counter[sg.t] = 0;
         }
-        named_bar_decoders();
+        named_bar_epilogue();
       }
+      PROF_ADD(1);
+      prof[2] += 1;
       ++seg;
-      x = seg_end;
+      x = sg.end;
     }
+    if (i == 64) PROF_FLUSH(40);
   }
 
   __syncthreads();
+  if (tid == 0 && p.trace) p.trace[blockIdx.x * 64 + 1] = clock64() - prof_start;
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);

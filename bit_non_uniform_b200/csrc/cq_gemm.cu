@@ -36,7 +36,8 @@ static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int epilogue, int sms
 }
 
 template <int NT>
-static int launch_engine(const EngineParams& p, const CUtensorMap& map, cudaStream_t s) {
+static int launch_engine(const EngineParams& p, const CUtensorMap& map, const CUtensorMap& wmap,
+                         cudaStream_t s) {
   using C = EngineCfg<NT>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -45,14 +46,15 @@ static int launch_engine(const EngineParams& p, const CUtensorMap& map, cudaStre
       return CQ_ERR_CUDA;
     attr_set = true;
   }
-  engine_kernel<NT><<<p.P, kThreads, C::SMEM, s>>>(p, map);
+  engine_kernel<NT><<<p.P, kThreads, C::SMEM, s>>>(p, map, wmap);
   return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
 }
 
 int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* scales,
               const uint16_t* ab, int64_t N, int64_t K, int B, int G, int grid_mode,
               int epilogue, int out_dtype, void* y, void* workspace, size_t ws_bytes,
-              cudaStream_t stream, uint64_t timeout_ns, int debug_skip) {
+              cudaStream_t stream, uint64_t timeout_ns, int debug_skip,
+              uint64_t* trace = nullptr) {
   int st = validate_matrix(packed, scales, ab, N, K, B, G, grid_mode);
   if (st != CQ_OK) return st;
   if (M < 0) return CQ_ERR_INVALID_ARG;
@@ -71,8 +73,10 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
   if (ws_bytes < need || (need && !workspace)) return CQ_ERR_WORKSPACE;
   if (!aligned(workspace, 16)) return CQ_ERR_UNSUPPORTED;
 
-  CUtensorMap map;
+  CUtensorMap map, wmap;
   st = encode_bf16_rows_sw128(&map, x, M, K, g.NT);
+  if (st != CQ_OK) return st;
+  st = encode_packed_rows(&wmap, packed, N, K * B / 8, B);
   if (st != CQ_OK) return st;
 
   EngineParams p = {};
@@ -98,12 +102,13 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
   p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + g.ws_counter_bytes);
   p.timeout_ns = timeout_ns;
   p.debug_skip_first_stage = debug_skip;
+  p.trace = trace;
 
   switch (g.NT) {
-    case 16: return launch_engine<16>(p, map, stream);
-    case 32: return launch_engine<32>(p, map, stream);
-    case 64: return launch_engine<64>(p, map, stream);
-    default: return launch_engine<128>(p, map, stream);
+    case 16: return launch_engine<16>(p, map, wmap, stream);
+    case 32: return launch_engine<32>(p, map, wmap, stream);
+    case 64: return launch_engine<64>(p, map, wmap, stream);
+    default: return launch_engine<128>(p, map, wmap, stream);
   }
 }
 
@@ -134,6 +139,19 @@ extern "C" int cq_gemm(const uint16_t* x, int64_t M, const uint8_t* packed, cons
                        void* stream) {
   return gemm_impl(x, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype, y,
                    workspace, ws_bytes, static_cast<cudaStream_t>(stream), kDefaultTimeoutNs, 0);
+}
+
+// Profiling hook (not part of the public header): cq_gemm that also writes
+// per-CTA event timestamps to trace ([grid][64] uint64, device memory, at
+// least cq_gemm_workspace_size-independent 148*64 entries).
+extern "C" CQ_API int cq_trace_gemm(const uint16_t* x, int64_t M, const uint8_t* packed,
+                                    const float* scales, const uint16_t* ab, int64_t N,
+                                    int64_t K, int B, int G, int epilogue, void* y,
+                                    void* workspace, size_t ws_bytes, uint64_t* trace,
+                                    void* stream) {
+  return gemm_impl(x, M, packed, scales, ab, N, K, B, G, CQ_GRID_MIDRISE, epilogue,
+                   CQ_DTYPE_F32, y, workspace, ws_bytes, static_cast<cudaStream_t>(stream),
+                   kDefaultTimeoutNs, 0, trace);
 }
 
 // Test hook (not part of the public header): run cq_gemm with a chosen wait

@@ -67,6 +67,26 @@ inline int encode_bf16_rows_sw128(CUtensorMap* map, const void* base, int64_t ro
   return r == CUDA_SUCCESS ? CQ_OK : CQ_ERR_CUDA;
 }
 
+// Tensor map over a packed CubicQuant matrix viewed as uint8 [rows][row_bytes],
+// loaded as boxes of 16*B bytes (one 128-code slice) x 64 rows.  The swizzle
+// (32-byte for B=2, 64-byte for B=4, none for B=3's 48-byte rows) keeps the
+// row-per-thread 16-byte shared-memory reads of the decoders conflict free.
+inline int encode_packed_rows(CUtensorMap* map, const void* base, int64_t rows,
+                              int64_t row_bytes, int B) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return CQ_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(16 * B), 64u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUtensorMapSwizzle sw = B == 2 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                 : (B == 4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE);
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CQ_OK : CQ_ERR_CUDA;
+}
+
 inline int num_sms() {
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
