@@ -72,6 +72,7 @@ def lib():
         "cq_moe_workspace_size": (sz, [i64, i32, i32, i64, i64, i32]),
         "cq_moe_grouped_gemm": (i32, [P, i64, P, P, i32, i32, P, i64, i64, i32, i32, i32,
                                       P, P, P, sz, P]),
+        "cq_gemm_noalloc": (i32, [P, i64, P, P, P, i64, i64, i32, i32, i32, i32, i32, P, P]),
         "cq_get_device_error": (i32, [P, ctypes.POINTER(ctypes.c_int)]),
         "cq_test_gemm_bounded": (i32, [P, i64, P, P, P, i64, i64, i32, i32, P, P, sz, u64,
                                        i32, P]),
@@ -158,6 +159,22 @@ def cq_gemm(x, packed, scales, ab, N: int, K: int, B: int, G: int, mode: int = M
                          epilogue, out_dtype, _ptr(out), _ptr(workspace),
                          workspace.numel() * workspace.element_size(), _stream(stream)),
            "cq_gemm")
+    return out
+
+
+def cq_gemm_noalloc(x, packed, scales, ab, N: int, K: int, B: int, G: int,
+                    mode: int = MIDRISE, epilogue: int = EPI_NONE, out_dtype: int = F32,
+                    out=None, stream=None):
+    """cq_gemm without a workspace (scratch in libcq's fixed array; M <= 16)."""
+    _need_cuda(x, packed, scales, ab)
+    M = x.shape[0]
+    ncol = N // 2 if epilogue == EPI_SWIGLU else N
+    if out is None:
+        dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+        out = torch.empty((M, ncol), dtype=dt, device=x.device)
+    _check(lib().cq_gemm_noalloc(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G,
+                                 mode, epilogue, out_dtype, _ptr(out), _stream(stream)),
+           "cq_gemm_noalloc")
     return out
 
 

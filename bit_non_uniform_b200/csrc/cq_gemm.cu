@@ -8,6 +8,8 @@
 
 namespace cq {
 
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;   // 2 s per wait
+
 static int pick_nt(int64_t M) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
@@ -121,8 +123,6 @@ size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int epilogue, int sm
 }  // namespace cq
 
 using namespace cq;
-
-static constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;   // 2 s per wait
 
 extern "C" size_t cq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int B, int G,
                                          int epilogue) {

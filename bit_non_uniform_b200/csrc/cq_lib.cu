@@ -3,3 +3,4 @@
 #include "cq_api.cu"
 #include "cq_gemm.cu"
 #include "cq_moe.cu"
+#include "cq_noalloc.cu"

@@ -125,6 +125,29 @@ CQ_API int cq_gemm(const uint16_t *x, int64_t M, const uint8_t *packed, const fl
             void *stream);
 
 /*
+ * cq_gemm_noalloc -- cq_gemm without a caller workspace, for callers that
+ * cannot allocate device memory: code that runs under an allocator it does
+ * not own (a plugin or operator inside another engine that hands it only
+ * inputs and outputs), or a latency-critical path whose memory is planned
+ * in advance and may not call cudaMalloc while serving.  Same arguments,
+ * semantics and results as cq_gemm (the article has no counterpart; this is
+ * a calling convenience).
+ *   Scratch: a fixed 4 MiB array inside libcq (every GPU that loads the
+ *   library holds it until the process exits), enough for any M <= 16 on a
+ *   148-SM B200; a problem that needs more returns CQ_ERR_WORKSPACE.
+ *   The first call on a device looks up that array's device address (a CUDA
+ *   runtime query) and caches it; make that first call before any stream
+ *   capture.  Every call shares the one array: calls that overlap on the GPU
+ *   (other streams, other host threads) race and must not be issued.
+ *   Each call clears the array's tile counters with cudaMemsetAsync on
+ *   `stream`; it calls no allocating routine.
+ */
+CQ_API int cq_gemm_noalloc(const uint16_t *x, int64_t M, const uint8_t *packed,
+                           const float *scales, const uint16_t *ab, int64_t N, int64_t K, int B,
+                           int G, int grid_mode, int epilogue, int out_dtype, void *y,
+                           void *stream);
+
+/*
  * One quantized matrix as seen by the grouped MoE call (device array).
  */
 typedef struct {
