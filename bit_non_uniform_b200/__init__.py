@@ -69,6 +69,8 @@ def lib():
         "cq_decode": (i32, [P, P, P, i64, i64, i32, i32, i32, i32, P, P]),
         "cq_gemm_workspace_size": (sz, [i64, i64, i64, i32, i32, i32]),
         "cq_gemm": (i32, [P, i64, P, P, P, i64, i64, i32, i32, i32, i32, i32, P, P, sz, P]),
+        "cq_moe_layer_bytes": (sz, [i32]),
+        "cq_moe_prepare_layer": (i32, [P, i32, i64, i64, i32, P]),
         "cq_moe_workspace_size": (sz, [i64, i32, i32, i64, i64, i32]),
         "cq_moe_grouped_gemm": (i32, [P, i64, P, P, i32, i32, P, i64, i64, i32, i32, i32,
                                       P, P, P, sz, P]),
@@ -182,10 +184,13 @@ def moe_workspace_size(T, k, E, H, I, G) -> int:
     return int(lib().cq_moe_workspace_size(T, k, E, H, I, G))
 
 
-def expert_table(experts, device="cuda"):
-    """Pack a list of per-expert dicts (gate_up / down packed, scales, ab, B)
-    into the device array of cq_expert_desc that cq_moe_grouped_gemm reads."""
-    arr = (ExpertDesc * len(experts))()
+def moe_prepare_layer(experts, H: int, I: int, G: int, device="cuda"):
+    """Build the device-side layer table (TMA descriptors + operand
+    descriptions) for a list of per-expert dicts with keys packed_gu,
+    scales_gu, ab_gu, B_gu, packed_dn, scales_dn, ab_dn, B_dn (CUDA tensors).
+    Returns the table (a uint8 CUDA tensor the caller keeps alive)."""
+    E = len(experts)
+    arr = (ExpertDesc * E)()
     for e, ex in enumerate(experts):
         for fld, key in (("gate_up", "gu"), ("down", "dn")):
             d = getattr(arr[e], fld)
@@ -194,16 +199,25 @@ def expert_table(experts, device="cuda"):
             d.ab = ex[f"ab_{key}"].data_ptr()
             d.B = int(ex[f"B_{key}"])
             d.reserved = 0
-    raw = bytes(arr)
-    host = torch.frombuffer(bytearray(raw), dtype=torch.uint8)
-    return host.to(device)
+    nbytes = int(lib().cq_moe_layer_bytes(E))
+    table = torch.empty(nbytes + 64, dtype=torch.uint8, device=device)
+    off = (-table.data_ptr()) % 64
+    table = table[off:off + nbytes]
+    _check(lib().cq_moe_prepare_layer(ctypes.cast(arr, ctypes.c_void_p), E, H, I, G,
+                                      _ptr(table)), "cq_moe_prepare_layer")
+    return table
 
 
-def cq_moe_grouped_gemm(tokens, topk_ids, topk_w, expert_descs, E: int, H: int, I: int,
-                        G: int, mode: int = MIDRISE, out_dtype: int = F32,
-                        route_out=True, combine=True, workspace=None, stream=None):
+def moe_workspace(T, k, E, H, I, G, device="cuda"):
+    n = moe_workspace_size(T, k, E, H, I, G)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def cq_moe_grouped_gemm(tokens, topk_ids, topk_w, layer, E: int, H: int, I: int, G: int,
+                        mode: int = MIDRISE, out_dtype: int = F32, route_out=True,
+                        combine=True, workspace=None, stream=None):
     """Routed-expert FFN of one MoE layer.  Returns (route_out, out)."""
-    _need_cuda(tokens, topk_ids, expert_descs)
+    _need_cuda(tokens, topk_ids, layer)
     T, k = topk_ids.shape
     ro = None
     if route_out is True:
@@ -215,11 +229,10 @@ def cq_moe_grouped_gemm(tokens, topk_ids, topk_w, expert_descs, E: int, H: int, 
         dt = torch.float32 if out_dtype == F32 else torch.bfloat16
         out = torch.empty((T, H), dtype=dt, device=tokens.device)
     if workspace is None:
-        n = moe_workspace_size(T, k, E, H, I, G)
-        workspace = torch.zeros(max(n, 16), dtype=torch.uint8, device=tokens.device)
+        workspace = moe_workspace(T, k, E, H, I, G, tokens.device)
     _check(lib().cq_moe_grouped_gemm(
         _ptr(tokens), T, _ptr(topk_ids), _ptr(topk_w) if topk_w is not None else None, k, E,
-        _ptr(expert_descs), H, I, G, mode, out_dtype, _ptr(ro), _ptr(out), _ptr(workspace),
+        _ptr(layer), H, I, G, mode, out_dtype, _ptr(ro), _ptr(out), _ptr(workspace),
         workspace.numel(), _stream(stream)), "cq_moe_grouped_gemm")
     return ro, out
 

@@ -77,6 +77,15 @@ struct MatrixRef {
   const float* scales;
   const uint32_t* ab;     // (a | b << 16), fp16 bits
   int B;
+  int reserved;
+};
+
+// One expert of a prepared MoE layer table (device memory, 64-byte aligned):
+// the TMA descriptors of its packed gate/up and down matrices, then their
+// operand descriptions.  Index 0 = gate/up [2I][H], 1 = down [H][I].
+struct alignas(64) LayerEntry {
+  CUtensorMap map[2];
+  MatrixRef mat[2];
 };
 
 struct EngineParams {
@@ -97,6 +106,16 @@ struct EngineParams {
   int n_tt;              // token tiles
   void* y;
   int64_t ldy;           // row stride of y in elements
+  // grouped (MoE) mode: tiles enumerate (active expert, row tile, token tile)
+  int grouped;
+  int which;                   // 0 = gate/up, 1 = down
+  const LayerEntry* layer;     // [E]
+  const int* g_ttpre;          // [E+1] prefix of token tiles per expert
+  const int* g_cnt;            // [E] routes per expert
+  const int* g_off;            // [E] first sorted route of each expert
+  const int* g_num_tiles;      // device scalar: tiles of this launch
+  const int* out_rows;         // optional sorted-position -> output row map
+  int E;
   // workspace
   float* partial;        // [2P][NT][128]
   int* counter;          // [num_tiles]
@@ -126,20 +145,51 @@ struct EngineParams {
 
 struct TileInfo {
   MatrixRef mat;
+  const CUtensorMap* wmap;   // TMA descriptor of the packed matrix
   int rt, tt;
   int x_row0;       // first activation row of the token tile (tensor map row)
   int m_valid;      // valid tokens in this tile (<= NT)
 };
 
-__device__ __forceinline__ TileInfo resolve_tile(const EngineParams& p, int t, int NT) {
+// Tile t of the launch.  Plain mode: t = rt * n_tt + tt.  Grouped mode:
+// experts in order, each contributing n_rt x ntt(e) tiles (tt fastest), so
+// expert e owns tiles [n_rt * ttpre[e], n_rt * ttpre[e+1]).
+__device__ __forceinline__ TileInfo resolve_tile(const EngineParams& p, int t, int NT,
+                                                 const CUtensorMap* plain_wmap) {
   TileInfo ti;
-  ti.mat = p.mat;
-  ti.rt = t / p.n_tt;
-  ti.tt = t - ti.rt * p.n_tt;
-  ti.x_row0 = ti.tt * NT;
-  const int rem = p.M - ti.x_row0;
+  if (!p.grouped) {
+    ti.mat = p.mat;
+    ti.wmap = plain_wmap;
+    ti.rt = t / p.n_tt;
+    ti.tt = t - ti.rt * p.n_tt;
+    ti.x_row0 = ti.tt * NT;
+    const int rem = p.M - ti.x_row0;
+    ti.m_valid = rem < NT ? rem : NT;
+    return ti;
+  }
+  // largest e with n_rt * ttpre[e] <= t (experts with no tiles are skipped)
+  int lo = 0, hi = p.E;                      // invariant: ttpre[lo]*n_rt <= t < ttpre[hi]*n_rt
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.n_rt * __ldg(p.g_ttpre + mid) <= t) lo = mid; else hi = mid;
+  }
+  const int e = lo;
+  const int ntt = __ldg(p.g_ttpre + e + 1) - __ldg(p.g_ttpre + e);
+  const int local = t - p.n_rt * __ldg(p.g_ttpre + e);
+  ti.rt = local / ntt;
+  ti.tt = local - ti.rt * ntt;
+  const LayerEntry* le = p.layer + e;
+  ti.mat = le->mat[p.which];
+  ti.wmap = &le->map[p.which];
+  ti.x_row0 = __ldg(p.g_off + e) + ti.tt * NT;
+  const int rem = __ldg(p.g_cnt + e) - ti.tt * NT;
   ti.m_valid = rem < NT ? rem : NT;
   return ti;
+}
+
+// Output row of sorted token position `pos`.
+__device__ __forceinline__ int64_t out_row(const EngineParams& p, int pos) {
+  return p.out_rows ? static_cast<int64_t>(__ldg(p.out_rows + pos)) : static_cast<int64_t>(pos);
 }
 
 // Global weight row of tile row i.
@@ -331,7 +381,7 @@ __device__ __forceinline__ void finalize16(const EngineParams& p, const TileInfo
         const int m = m0 + q;
         if (m < ti.m_valid) {
           const float h = silu_f(v[q]) * xchg[q * 64 + i];
-          const int64_t off = static_cast<int64_t>(ti.x_row0 + m) * p.ldy + col;
+          const int64_t off = out_row(p, ti.x_row0 + m) * p.ldy + col;
           if (p.out_bf16)
             reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(h);
           else
@@ -346,7 +396,7 @@ __device__ __forceinline__ void finalize16(const EngineParams& p, const TileInfo
       for (int q = 0; q < 16; ++q) {
         const int m = m0 + q;
         if (m < ti.m_valid) {
-          const int64_t off = static_cast<int64_t>(ti.x_row0 + m) * p.ldy + grow;
+          const int64_t off = out_row(p, ti.x_row0 + m) * p.ldy + grow;
           if (p.out_bf16)
             reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(v[q]);
           else
@@ -424,16 +474,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 4 && lane == 0) {
     prefetch_tensormap(&xmap);
-    prefetch_tensormap(&wmap);
+    if (!p.grouped) prefetch_tensormap(&wmap);
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base =
       *reinterpret_cast<volatile uint32_t*>(gbase + (slot_tmem - base));
 
-  const int64_t W = static_cast<int64_t>(p.num_tiles) * p.spt;
-  const int64_t r0 = range_begin(W, p.P, cta);
-  const int64_t r1 = range_begin(W, p.P, cta + 1);
+  const int num_tiles = p.grouped ? *reinterpret_cast<const volatile int*>(p.g_num_tiles)
+                                  : p.num_tiles;
+  const int64_t W = static_cast<int64_t>(num_tiles) * p.spt;
+  // CTAs that take part: at most one per slice, so that every CTA of the
+  // partition owns at least one slice (the stream-K reduction counts on it)
+  const int Pe = W < p.P ? static_cast<int>(W) : p.P;
+  const int64_t r0 = cta < Pe ? range_begin(W, Pe, cta) : W;
+  const int64_t r1 = cta < Pe ? range_begin(W, Pe, cta + 1) : W;
   const uint64_t tmo = p.timeout_ns;
 
   if (warp == 4) {
@@ -443,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int load_no = 0;
     for (int64_t x = r0; x < r1 && !*abort_flag;) {
       const Segment sg = segment_at(x, r1, p.spt);
-      const TileInfo ti = resolve_tile(p, sg.t, NT);
+      const TileInfo ti = resolve_tile(p, sg.t, NT, &wmap);
       const int Bw = ti.mat.B;
       // first weight row of the two 64-row boxes of this tile
       const int row_a = tile_row(p, ti.rt, 0);
@@ -466,8 +521,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < ns; ++j) {
             const int cb = (sb + j) * 16 * Bw;                   // byte column of the slice
             const uint32_t sdst = wdst + j * C::SLICE_W_BYTES;
-            tma_load_2d(sdst, &wmap, cb, row_a, bar_full + 8 * st);
-            tma_load_2d(sdst + wbox, &wmap, cb, row_b, bar_full + 8 * st);
+            tma_load_2d(sdst, ti.wmap, cb, row_a, bar_full + 8 * st);
+            tma_load_2d(sdst + wbox, ti.wmap, cb, row_b, bar_full + 8 * st);
           }
           for (int b = 0; b < 2 * ns; ++b)
             tma_load_2d(xdst + b * (NT * 128), &xmap, sb * kSlice + b * 64, ti.x_row0,
@@ -585,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ng = p.K / p.G;
     for (int64_t x = r0; ok && x < r1;) {
       const Segment sg = segment_at(x, r1, p.spt);
-      const TileInfo ti = resolve_tile(p, sg.t, NT);
+      const TileInfo ti = resolve_tile(p, sg.t, NT, &wmap);
       const int Bw = ti.mat.B;
       const int grow = tile_row(p, ti.rt, i);
       // 16-byte chunk v of this row sits at chunk (v ^ swz) of the row (TMA swizzle)
@@ -676,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int64_t x = r0; ok && x < r1;) {
       const Segment sg = segment_at(x, r1, p.spt);
-      const TileInfo ti = resolve_tile(p, sg.t, NT);
+      const TileInfo ti = resolve_tile(p, sg.t, NT, &wmap);
       const int grow = tile_row(p, ti.rt, i);
       const uint32_t db = seg & 1u;
       PROF_MARK();
@@ -720,8 +775,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar_dfree + 8 * db);
         __threadfence();
         named_bar_epilogue();
-        const int c_lo = owner_of(W, p.P, static_cast<int64_t>(sg.t) * p.spt);
-        const int c_hi = owner_of(W, p.P, static_cast<int64_t>(sg.t) * p.spt + p.spt - 1);
+        const int c_lo = owner_of(W, Pe, static_cast<int64_t>(sg.t) * p.spt);
+        const int c_hi = owner_of(W, Pe, static_cast<int64_t>(sg.t) * p.spt + p.spt - 1);
         if (i == 0) {
           const int old = atomicAdd(p.counter + sg.t, 1);
           *last_flag = (old == c_hi - c_lo) ? 1 : 0;
@@ -735,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 16; ++k) v[k] = 0.f;
             for (int c = c_lo; c <= c_hi; ++c) {
-              const int ft = static_cast<int>(range_begin(W, p.P, c) / p.spt);
+              const int ft = static_cast<int>(range_begin(W, Pe, c) / p.spt);
               const int sl = 2 * c + (sg.t == ft ? 0 : 1);
               const float* src = p.partial + static_cast<int64_t>(sl) * NT * kRows;
 #pragma unroll

@@ -148,7 +148,7 @@ CQ_API int cq_gemm_noalloc(const uint16_t *x, int64_t M, const uint8_t *packed,
                            void *stream);
 
 /*
- * One quantized matrix as seen by the grouped MoE call (device array).
+ * One quantized matrix of an expert (HOST-side description, device pointers).
  */
 typedef struct {
     const uint8_t *packed;   /* [rows][cols*B/8]        */
@@ -164,26 +164,44 @@ typedef struct {
 } cq_expert_desc;
 
 /*
+ * cq_moe_prepare_layer -- build the device-side table of one MoE layer:
+ * for each of the E experts, the TMA descriptors of its packed gate/up and
+ * down matrices and their operand descriptions.  `experts` is a HOST array
+ * of E descriptions (device pointers inside); `layer` is device memory of
+ * cq_moe_layer_bytes(E) bytes owned by the caller, valid as long as the
+ * expert weights do not move.  Synchronous (run once per layer, at load).
+ * Each matrix must satisfy the cq_gemm requirements (B in {2,3,4},
+ * G % 128 == 0, H and I multiples of G, I % 64 == 0, packed 16-byte aligned).
+ */
+CQ_API size_t cq_moe_layer_bytes(int E);
+CQ_API int cq_moe_prepare_layer(const cq_expert_desc *experts, int E, int64_t H, int64_t I,
+                                int G, void *layer);
+
+/*
  * cq_moe_grouped_gemm -- the routed-expert FFN of one MoE layer, with
  * per-expert CubicQuant weights (the quantized tensors of [CQ] are the
- * routed experts, section "先看结论").  For every route r = (t, j):
+ * routed experts, section "先看结论").  For every route r = t*k + j:
  *   e = topk_ids[t][j];  g|u = W_gu[e] x_t;  h = bf16(silu(g) * u);
  *   y_r = W_dn[e] h  (FP32 accumulation)
- * and, when out != NULL, out[t] = sum_j topk_w[t][j] * y_(t,j) (j ascending).
+ * and, when out != NULL, out[t] = sum_j topk_w[t][j] * y_(t,j) (j ascending,
+ * FP32).  Routing is done on the device (no host synchronisation): routes
+ * are grouped by expert, then one grouped launch runs every active expert's
+ * gate/up tiles with the SwiGLU epilogue and one runs the down tiles.
  *   tokens     bfloat16 [T][H]
- *   topk_ids   int32 [T][k], values in [0, E)
+ *   topk_ids   int32 [T][k]; an id outside [0, E) drops that route (its
+ *              y_r is zero) and is counted in the device error word
  *   topk_w     float [T][k] (required when out != NULL)
- *   experts    device array of E cq_expert_desc
+ *   layer      table built by cq_moe_prepare_layer for these E experts
  *   route_out  float [T*k][H] per-route outputs y_r (may be NULL)
  *   out        [T][H] combined output in out_dtype (may be NULL)
- * Requires H and I multiples of G, G % 128 == 0, I % 64 == 0.
+ *   workspace  device scratch of at least cq_moe_workspace_size(...) bytes
+ * Calls that share one workspace must not overlap on the GPU.
  */
 CQ_API size_t cq_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I, int G);
 CQ_API int cq_moe_grouped_gemm(const uint16_t *tokens, int64_t T, const int32_t *topk_ids,
-                        const float *topk_w, int k, int E,
-                        const cq_expert_desc *experts, int64_t H, int64_t I, int G,
-                        int grid_mode, int out_dtype, void *route_out, void *out,
-                        void *workspace, size_t ws_bytes, void *stream);
+                               const float *topk_w, int k, int E, const void *layer, int64_t H,
+                               int64_t I, int G, int grid_mode, int out_dtype, void *route_out,
+                               void *out, void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * cq_get_device_error -- synchronise `stream`, then read and clear the

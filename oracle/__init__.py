@@ -221,7 +221,7 @@ def bf16_bits_to_f64(h: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------
 
 def moe_routes(tokens_bf16bits, topk_ids, experts, H, I, G, mode=MIDRISE,
-               routes=None, nthreads=0):
+               routes=None, nthreads=0, rel=2e-3, abs_=1e-6):
     """Per-route outputs of the routed-expert FFN, FP64.
 
     experts[e] = dict(B_gu, packed_gu [2I][H*B/8], scales_gu, ab_gu,
@@ -233,7 +233,16 @@ def moe_routes(tokens_bf16bits, topk_ids, experts, H, I, G, mode=MIDRISE,
         y_r = W_dn h (H outputs).
     h is rounded to BF16 because the GPU chain stores it in BF16.
     routes: optional list of flat route indices r = t*k + j to evaluate.
-    Returns dict r -> (y_r [H] float64, bound_r [H] float64)."""
+
+    Returns dict r -> (y_r, bound_r, tol_r), all [H] float64:
+      bound_r = sum_i |w_dn[n][i] h_i|;
+      tol_r   = the per-GEMM tolerance rel*bound + abs_ of the down product
+                plus the first-order effect of the gate/up product's own
+                tolerance on h: each g, u may be off by e = rel*sum|w x| +
+                abs_, which moves h = silu(g) u by at most
+                |silu'(g)| |u| e_g + |silu(g)| e_u + e_g e_u, and the BF16
+                rounding of a perturbed h may land one BF16 ulp (<= 2^-7 |h|)
+                away; that input difference reaches y_r through |W_dn|."""
     T, k = topk_ids.shape
     if routes is None:
         routes = range(T * k)
@@ -247,13 +256,24 @@ def moe_routes(tokens_bf16bits, topk_ids, experts, H, I, G, mode=MIDRISE,
         rs = by_expert[e]
         ex = get(e)
         xs = np.ascontiguousarray(tokens_bf16bits[[r // k for r in rs]])
-        gu, _ = gemm(xs, ex["packed_gu"], ex["scales_gu"], ex["ab_gu"], 2 * I, H,
-                     ex["B_gu"], G, mode, nthreads)
-        h = bf16_round(swiglu(gu))
-        y, bnd = gemm(h, ex["packed_dn"], ex["scales_dn"], ex["ab_dn"], H, I,
+        gu, bgu = gemm(xs, ex["packed_gu"], ex["scales_gu"], ex["ab_gu"], 2 * I, H,
+                       ex["B_gu"], G, mode, nthreads)
+        hf = swiglu(gu)
+        hb = bf16_round(hf)
+        h = bf16_bits_to_f64(hb)
+        y, bnd = gemm(hb, ex["packed_dn"], ex["scales_dn"], ex["ab_dn"], H, I,
                       ex["B_dn"], G, mode, nthreads)
+        g, u = gu[:, :I], gu[:, I:]
+        eg, eu = rel * bgu[:, :I] + abs_, rel * bgu[:, I:] + abs_
+        sig = 1.0 / (1.0 + np.exp(-g))
+        dsilu = np.abs(sig * (1.0 + g * (1.0 - sig)))
+        eh = dsilu * np.abs(u) * eg + np.abs(g * sig) * eu + eg * eu + 1e-6 * np.abs(hf)
+        dh = eh + 2.0 ** -7 * (np.abs(h) + eh)
+        wdn, _, _ = decode(ex["packed_dn"], ex["scales_dn"], ex["ab_dn"], H, I, ex["B_dn"], G,
+                           mode)
+        prop = dh @ np.abs(wdn).T
         for i, r in enumerate(rs):
-            out[r] = (y[i], bnd[i])
+            out[r] = (y[i], bnd[i], rel * bnd[i] + abs_ + prop[i])
     return out
 
 
@@ -267,7 +287,7 @@ def moe_combine(route_out, topk_w, tokens=None):
         acc = None
         bnd = None
         for j in range(k):
-            y, b = route_out[t * k + j]
+            y, b = route_out[t * k + j][:2]
             w = float(topk_w[t, j])
             acc = w * y if acc is None else acc + w * y
             bnd = abs(w) * b if bnd is None else bnd + abs(w) * b

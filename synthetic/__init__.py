@@ -78,7 +78,9 @@ def make_key(*tags) -> int:
     """Mix integer / string tags into one 64-bit key."""
     k = 0x5EED
     for t in tags:
-        if isinstance(t, str):
+        if isinstance(t, (tuple, list)):
+            t = make_key(*t)
+        elif isinstance(t, str):
             t = int.from_bytes(t.encode(), "little") & _MASK64
         k = splitmix64_py(k ^ (int(t) & _MASK64), 0)
     return k
