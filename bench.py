@@ -241,6 +241,81 @@ def time_gemm(cq, name, steps, warmup, world, device, sample_clocks=False):
     return res
 
 
+MOE_WORKLOADS = {
+    # name: (description, T, routing, widths)
+    "moe_decode": ("Kimi-K3 MoE layer, 896 experts W2/W3/W4 (P=.6/.3/.1) G512, 64 tokens, "
+                   "uniform top-16", 64, "uniform", "mixed"),
+    "moe_prefill": ("Kimi-K3 MoE layer, 896 experts W4 G512, 8192 tokens, Zipf(1.1) top-16",
+                    8192, "zipf", "w4"),
+}
+
+
+def time_moe(cq, name, steps, device):
+    """Device-timed steps of one MoE layer (routing, gather, gate/up, down,
+    combine), captured in a CUDA graph; inputs and weights resident."""
+    import synthetic
+    desc, T, routing, widths = MOE_WORKLOADS[name]
+    H, I, E, k, G = 7168, 3072, 896, 16, 512
+    Bs = synthetic.expert_bits(4, E) if widths == "mixed" else torch.full((E,), 4)
+    experts = []
+    for e in range(E):
+        B = int(Bs[e])
+        gu = synthetic.matrix(("bench", name, "gu", e), 2 * I, H, B, G, device=device)
+        dn = synthetic.matrix(("bench", name, "dn", e), H, I, B, G, device=device)
+        experts.append(dict(B_gu=B, packed_gu=cq.cq_pack(gu[0], B), scales_gu=gu[1],
+                            ab_gu=gu[2], B_dn=B, packed_dn=cq.cq_pack(dn[0], B),
+                            scales_dn=dn[1], ab_dn=dn[2]))
+        del gu, dn
+    layer = cq.moe_prepare_layer(experts, H, I, G, device)
+    x = synthetic.activations(7, T, H).to(device)
+    if routing == "uniform":
+        ids, w = synthetic.routing_uniform(4, T, E, k)
+    else:
+        ids, w = synthetic.routing_zipf(5, T, E, k)
+    ids_d, w_d = ids.to(device), w.to(device)
+    ws = cq.moe_workspace(T, k, E, H, I, G, device)
+    out = torch.empty((T, H), dtype=torch.float32, device=device)
+    stream = torch.cuda.Stream(device)
+    lib = cq.lib()
+
+    def step():
+        st = lib.cq_moe_grouped_gemm(
+            cq._ptr(x), T, cq._ptr(ids_d), cq._ptr(w_d), k, E, cq._ptr(layer), H, I, G, 0, 0,
+            None, cq._ptr(out), cq._ptr(ws), ws.numel(), cq._stream(stream))
+        if st != 0:
+            raise RuntimeError(f"cq_moe_grouped_gemm status {st}")
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(steps):
+            step()
+    g.replay()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+    ev1.record(stream)
+    ev1.synchronize()
+    ms = ev0.elapsed_time(ev1) / steps
+    st, site = cq.device_error()
+    if st != 0:
+        raise RuntimeError(f"device wait timed out (site {site})")
+    del g
+    active = torch.unique(ids).tolist()
+    wbytes = sum(packed_bytes(2 * I, H, int(Bs[e]), G) + packed_bytes(H, I, int(Bs[e]), G)
+                 for e in active)
+    flops = 2.0 * T * k * (2 * I * H + H * I)
+    mean_bits = sum(int(Bs[e]) for e in active) / len(active)
+    return dict(name=name, desc=desc, ms=ms, tokens_per_s=T / (ms * 1e-3),
+                gbs=wbytes / (ms * 1e-3) / 1e9, tflops=flops / (ms * 1e-3) / 1e12,
+                active=len(active), wbytes=wbytes, mean_payload_bits=mean_bits)
+
+
 class _null:
     def __enter__(self):
         return self
@@ -370,6 +445,7 @@ def main():
     ap.add_argument("--workload", default="down_m1", choices=sorted(WORKLOADS))
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-moe", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -406,6 +482,27 @@ def main():
                                    "peak": tf_burst, "unit": "TFLOP/s",
                                    "frac": round(r["tflops"] / tf_burst, 4)}
             secondary.append(ent)
+
+    if not args.no_secondary and not args.no_moe:
+        for name in ["moe_decode", "moe_prefill"]:
+            r = time_moe(cq, name, 20 if name == "moe_decode" else 5, device)
+            ent = {"workload": r["desc"], "ms_per_step": round(r["ms"], 4),
+                   "tokens_per_s": round(r["tokens_per_s"] * world, 1),
+                   "packed_gbs": round(r["gbs"] * world, 1),
+                   "tflops": round(r["tflops"] * world, 2),
+                   "active_experts": r["active"],
+                   "active_weight_bytes": r["wbytes"],
+                   "mean_payload_bits_active": round(r["mean_payload_bits"], 4)}
+            if name == "moe_decode":
+                ent["roofline"] = {"bound": "hbm", "achieved": round(r["gbs"], 1), "peak": hbm,
+                                   "unit": "GB/s", "frac": round(r["gbs"] / hbm, 4)}
+            else:
+                ent["roofline"] = {"bound": "tensor", "achieved": round(r["tflops"], 1),
+                                   "peak": tf_sust, "unit": "TFLOP/s",
+                                   "frac": round(r["tflops"] / tf_sust, 4),
+                                   "peak_kind": "sustained"}
+            secondary.append(ent)
+            torch.cuda.empty_cache()
 
     e2e = time_e2e(cq, args.workload, args.steps, device)
     e2e["value"] = round(e2e["value"] * world, 3)

@@ -119,6 +119,10 @@ struct EngineParams {
   // workspace
   float* partial;        // [2P][NT][128]
   int* counter;          // [num_tiles]
+  // extents of the buffers above, checked before every global access
+  int64_t y_rows;        // rows of y
+  int partial_slots;     // slots of partial
+  int counter_len;       // entries of counter
   // control
   uint64_t timeout_ns;
   int debug_skip_first_stage;   // test hook: never issue stage load 0
@@ -143,9 +147,21 @@ struct EngineParams {
       for (int k_ = 0; k_ < 8; ++k_) p.trace[blockIdx.x * 64 + (base) + k_] = prof[k_]; \
   } while (0)
 
+// Load through a pointer that is null in plain mode.  The volatile asm can
+// neither be hoisted above the branch that guards it nor turned into an
+// unconditional load by if-conversion.
+__device__ __forceinline__ int ld_guarded(const int* ptr) {
+  int v;
+  asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(ptr));
+  return v;
+}
+
+// Record a failed bounds check (site >= 20) in the device error word.
+__device__ __forceinline__ void bad_access(int site) { atomicCAS(&g_device_error, 0, site); }
+
 struct TileInfo {
   MatrixRef mat;
-  const CUtensorMap* wmap;   // TMA descriptor of the packed matrix
+  const CUtensorMap* wmap;   // grouped mode: the expert's TMA descriptor (global memory)
   int rt, tt;
   int x_row0;       // first activation row of the token tile (tensor map row)
   int m_valid;      // valid tokens in this tile (<= NT)
@@ -154,12 +170,11 @@ struct TileInfo {
 // Tile t of the launch.  Plain mode: t = rt * n_tt + tt.  Grouped mode:
 // experts in order, each contributing n_rt x ntt(e) tiles (tt fastest), so
 // expert e owns tiles [n_rt * ttpre[e], n_rt * ttpre[e+1]).
-__device__ __forceinline__ TileInfo resolve_tile(const EngineParams& p, int t, int NT,
-                                                 const CUtensorMap* plain_wmap) {
+__device__ __forceinline__ TileInfo resolve_tile(const EngineParams& p, int t, int NT) {
   TileInfo ti;
   if (!p.grouped) {
     ti.mat = p.mat;
-    ti.wmap = plain_wmap;
+    ti.wmap = nullptr;          // plain mode loads through the kernel's own parameter
     ti.rt = t / p.n_tt;
     ti.tt = t - ti.rt * p.n_tt;
     ti.x_row0 = ti.tt * NT;
@@ -171,25 +186,27 @@ __device__ __forceinline__ TileInfo resolve_tile(const EngineParams& p, int t, i
   int lo = 0, hi = p.E;                      // invariant: ttpre[lo]*n_rt <= t < ttpre[hi]*n_rt
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (p.n_rt * __ldg(p.g_ttpre + mid) <= t) lo = mid; else hi = mid;
+    if (p.n_rt * ld_guarded(p.g_ttpre + mid) <= t) lo = mid; else hi = mid;
   }
   const int e = lo;
-  const int ntt = __ldg(p.g_ttpre + e + 1) - __ldg(p.g_ttpre + e);
-  const int local = t - p.n_rt * __ldg(p.g_ttpre + e);
+  if (e < 0 || e >= p.E) bad_access(26);
+  const int ntt = ld_guarded(p.g_ttpre + e + 1) - ld_guarded(p.g_ttpre + e);
+  const int local = t - p.n_rt * ld_guarded(p.g_ttpre + e);
   ti.rt = local / ntt;
   ti.tt = local - ti.rt * ntt;
   const LayerEntry* le = p.layer + e;
   ti.mat = le->mat[p.which];
   ti.wmap = &le->map[p.which];
-  ti.x_row0 = __ldg(p.g_off + e) + ti.tt * NT;
-  const int rem = __ldg(p.g_cnt + e) - ti.tt * NT;
+  ti.x_row0 = ld_guarded(p.g_off + e) + ti.tt * NT;
+  const int rem = ld_guarded(p.g_cnt + e) - ti.tt * NT;
   ti.m_valid = rem < NT ? rem : NT;
   return ti;
 }
 
 // Output row of sorted token position `pos`.
 __device__ __forceinline__ int64_t out_row(const EngineParams& p, int pos) {
-  return p.out_rows ? static_cast<int64_t>(__ldg(p.out_rows + pos)) : static_cast<int64_t>(pos);
+  if (p.out_rows) return static_cast<int64_t>(ld_guarded(p.out_rows + pos));
+  return static_cast<int64_t>(pos);
 }
 
 // Global weight row of tile row i.
@@ -381,8 +398,11 @@ __device__ __forceinline__ void finalize16(const EngineParams& p, const TileInfo
         const int m = m0 + q;
         if (m < ti.m_valid) {
           const float h = silu_f(v[q]) * xchg[q * 64 + i];
-          const int64_t off = out_row(p, ti.x_row0 + m) * p.ldy + col;
-          if (p.out_bf16)
+          const int64_t orow = out_row(p, ti.x_row0 + m);
+          const int64_t off = orow * p.ldy + col;
+          if (orow < 0 || orow >= p.y_rows || col >= p.ldy) {
+            bad_access(23);
+          } else if (p.out_bf16)
             reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(h);
           else
             reinterpret_cast<float*>(p.y)[off] = h;
@@ -396,8 +416,11 @@ __device__ __forceinline__ void finalize16(const EngineParams& p, const TileInfo
       for (int q = 0; q < 16; ++q) {
         const int m = m0 + q;
         if (m < ti.m_valid) {
-          const int64_t off = out_row(p, ti.x_row0 + m) * p.ldy + grow;
-          if (p.out_bf16)
+          const int64_t orow = out_row(p, ti.x_row0 + m);
+          const int64_t off = orow * p.ldy + grow;
+          if (orow < 0 || orow >= p.y_rows || grow >= p.ldy) {
+            bad_access(23);
+          } else if (p.out_bf16)
             reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(v[q]);
           else
             reinterpret_cast<float*>(p.y)[off] = v[q];
@@ -481,8 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base =
       *reinterpret_cast<volatile uint32_t*>(gbase + (slot_tmem - base));
 
-  const int num_tiles = p.grouped ? *reinterpret_cast<const volatile int*>(p.g_num_tiles)
-                                  : p.num_tiles;
+  int num_tiles = p.num_tiles;
+  if (p.grouped) num_tiles = ld_guarded(p.g_num_tiles);
   const int64_t W = static_cast<int64_t>(num_tiles) * p.spt;
   // CTAs that take part: at most one per slice, so that every CTA of the
   // partition owns at least one slice (the stream-K reduction counts on it)
@@ -498,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int load_no = 0;
     for (int64_t x = r0; x < r1 && !*abort_flag;) {
       const Segment sg = segment_at(x, r1, p.spt);
-      const TileInfo ti = resolve_tile(p, sg.t, NT, &wmap);
+      const TileInfo ti = resolve_tile(p, sg.t, NT);
       const int Bw = ti.mat.B;
       // first weight row of the two 64-row boxes of this tile
       const int row_a = tile_row(p, ti.rt, 0);
@@ -511,7 +534,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         PROF_ADD(0);
         const bool skip = p.debug_skip_first_stage && load_no == 0;
-        if (!skip && lane == 0) {
+        // the kernel parameter's address is only ever used directly in the
+        // TMA instruction; table descriptors must lie inside the table
+        const bool map_ok =
+            !p.grouped || (ti.wmap >= &p.layer[0].map[0] && ti.wmap < &p.layer[p.E].map[0]);
+        if (!map_ok && lane == 0) bad_access(21);
+        if (!skip && map_ok && lane == 0) {
           const uint32_t wbox = 64u * 16u * Bw;                   // bytes of one weight box
           const uint32_t bytes = static_cast<uint32_t>(ns) * (2u * wbox) +
                                  static_cast<uint32_t>(2 * ns * NT * 128);
@@ -521,8 +549,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < ns; ++j) {
             const int cb = (sb + j) * 16 * Bw;                   // byte column of the slice
             const uint32_t sdst = wdst + j * C::SLICE_W_BYTES;
-            tma_load_2d(sdst, ti.wmap, cb, row_a, bar_full + 8 * st);
-            tma_load_2d(sdst + wbox, ti.wmap, cb, row_b, bar_full + 8 * st);
+            if (p.grouped) {
+              tma_load_2d(sdst, ti.wmap, cb, row_a, bar_full + 8 * st);
+              tma_load_2d(sdst + wbox, ti.wmap, cb, row_b, bar_full + 8 * st);
+            } else {
+              tma_load_2d(sdst, &wmap, cb, row_a, bar_full + 8 * st);
+              tma_load_2d(sdst + wbox, &wmap, cb, row_b, bar_full + 8 * st);
+            }
           }
           for (int b = 0; b < 2 * ns; ++b)
             tma_load_2d(xdst + b * (NT * 128), &xmap, sb * kSlice + b * 64, ti.x_row0,
@@ -640,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ng = p.K / p.G;
     for (int64_t x = r0; ok && x < r1;) {
       const Segment sg = segment_at(x, r1, p.spt);
-      const TileInfo ti = resolve_tile(p, sg.t, NT, &wmap);
+      const TileInfo ti = resolve_tile(p, sg.t, NT);
       const int Bw = ti.mat.B;
       const int grow = tile_row(p, ti.rt, i);
       // 16-byte chunk v of this row sits at chunk (v ^ swz) of the row (TMA swizzle)
@@ -651,9 +684,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int g_next = (sg.s0 * kSlice) / p.G;
       float s_next = 0.f;
       uint32_t ab_next = 0;
-      if (valid) {
+      if (valid && g_next < ng) {
         s_next = __ldg(ti.mat.scales + static_cast<int64_t>(grow) * ng + g_next);
         ab_next = __ldg(ti.mat.ab + static_cast<int64_t>(grow) * ng + g_next);
+      } else if (valid) {
+        bad_access(22);
       }
       for (int sb = sg.s0; sb < sg.s1 && ok; sb += C::SPS) {
         const int ns = (sg.s1 - sb) < C::SPS ? (sg.s1 - sb) : C::SPS;
@@ -731,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int64_t x = r0; ok && x < r1;) {
       const Segment sg = segment_at(x, r1, p.spt);
-      const TileInfo ti = resolve_tile(p, sg.t, NT, &wmap);
+      const TileInfo ti = resolve_tile(p, sg.t, NT);
       const int grow = tile_row(p, ti.rt, i);
       const uint32_t db = seg & 1u;
       PROF_MARK();
@@ -762,14 +797,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // partial tile: park it in the workspace, the last contributor reduces
         const int first_tile = static_cast<int>(r0 / p.spt);
         const int slot = 2 * cta + (sg.t == first_tile ? 0 : 1);
-        float* const mine = p.partial + static_cast<int64_t>(slot) * NT * kRows;
+        const bool slot_ok = slot < p.partial_slots && sg.t < p.counter_len;
+        if (!slot_ok && i == 0) bad_access(24);
+        float* const mine = p.partial + static_cast<int64_t>(slot_ok ? slot : 0) * NT * kRows;
         for (int cc = 0; cc < nchunks; ++cc) {
           uint32_t rr[16];
           tmem_ld16(daddr + cc * 16, rr);
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 16; ++k)
-            if (cc * 16 + k < ti.m_valid) mine[(cc * 16 + k) * kRows + i] = __uint_as_float(rr[k]);
+            if (slot_ok && cc * 16 + k < ti.m_valid)
+              mine[(cc * 16 + k) * kRows + i] = __uint_as_float(rr[k]);
         }
         tc_fence_before();
         mbar_arrive(bar_dfree + 8 * db);
@@ -778,7 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c_lo = owner_of(W, Pe, static_cast<int64_t>(sg.t) * p.spt);
         const int c_hi = owner_of(W, Pe, static_cast<int64_t>(sg.t) * p.spt + p.spt - 1);
         if (i == 0) {
-          const int old = atomicAdd(p.counter + sg.t, 1);
+          const int old = slot_ok ? atomicAdd(p.counter + sg.t, 1) : -1;
           *last_flag = (old == c_hi - c_lo) ? 1 : 0;
         }
         named_bar_epilogue();
@@ -792,6 +830,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = c_lo; c <= c_hi; ++c) {
               const int ft = static_cast<int>(range_begin(W, Pe, c) / p.spt);
               const int sl = 2 * c + (sg.t == ft ? 0 : 1);
+              if (sl >= p.partial_slots) {
+                bad_access(25);
+                continue;
+              }
               const float* src = p.partial + static_cast<int64_t>(sl) * NT * kRows;
 #pragma unroll
               for (int k = 0; k < 16; ++k)
@@ -799,7 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             finalize16(p, ti, i, grow, v, cc, xchg);
           }
-          if (i == 0) p.counter[sg.t] = 0;
+          if (i == 0 && slot_ok) p.counter[sg.t] = 0;
         }
         named_bar_epilogue();
       }

@@ -100,6 +100,9 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
   p.n_tt = g.n_tt;
   p.y = y;
   p.ldy = epilogue == CQ_EPI_SWIGLU ? N / 2 : N;
+  p.y_rows = M;
+  p.partial_slots = 2 * g.P;
+  p.counter_len = g.tiles;
   p.counter = reinterpret_cast<int*>(workspace);
   p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + g.ws_counter_bytes);
   p.timeout_ns = timeout_ns;

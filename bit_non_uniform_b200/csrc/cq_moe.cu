@@ -377,6 +377,9 @@ extern "C" int cq_moe_grouped_gemm(const uint16_t* tokens, int64_t T, const int3
     p.ldy = which == 0 ? I : H;
     p.partial = part;
     p.counter = which == 0 ? cgu : cdn;
+    p.y_rows = m.R;
+    p.partial_slots = 2 * m.P;
+    p.counter_len = static_cast<int>((which == 0 ? m.n_rt_gu : m.n_rt_dn) * m.max_tt);
     p.timeout_ns = kDefaultTimeoutNs;
     st = launch_grouped_nt(m.NT, p, which == 0 ? xmap_gu : xmap_dn, s);
     if (st != CQ_OK) return st;
