@@ -26,6 +26,7 @@ enum WaitSite : int {
   SITE_MMA_AREADY = 6,
   SITE_MMA_DFREE = 7,
   SITE_TEARDOWN = 8,
+  SITE_TABLE = 9,
 };
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -76,6 +77,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread for up to hint_ns
+// (it wakes as soon as the phase completes), so waiting warps do not take
+// issue slots from the warps doing work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Gives up after
 // timeout_ns (or as soon as *abort is set by another thread), records the
 // site in the CTA abort flag and the device error word, and returns false.
@@ -84,7 +101,7 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*abort) return false;
     if (globaltimer() - t0 > timeout_ns) {
       *abort = site;

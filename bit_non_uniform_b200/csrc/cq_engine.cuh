@@ -9,24 +9,25 @@
 // epilogue.
 //
 // Warp roles (320 threads):
-//   warps 0-3  decoders: thread i owns weight row i of the tile and TMEM
-//              lane i.  Per group it builds a private BF16 pair table
-//              (two codes -> two levels, one 32-bit word per entry, the
-//              entries of all 128 threads interleaved so that every lookup
-//              hits the thread's own bank), then turns each slice of packed
-//              codes into 64 BF16x2 words written to TMEM with tcgen05.st
+//   warps 0-7  decoders: weight row i of the tile (TMEM lane i) belongs to
+//              thread i%32 of warps i/32 and i/32+4.  Per group the two
+//              build the row's BF16 pair table (two codes -> two levels,
+//              one 32-bit word per entry, the entries of all 128 rows
+//              interleaved so that every lookup of a warp hits 32 distinct
+//              banks) half each, then each turns its half of every 128-code
+//              slice into 32 BF16x2 words written to TMEM with tcgen05.st
 //              (the A operand of the MMA).
-//   warp 4     producer: 2-D TMA loads into a ring of shared-memory
+//   warp 8     producer: 2-D TMA loads into a ring of shared-memory
 //              stages: per 128-code slice, two boxes of 64 weight rows x
 //              16*B bytes of packed codes (32-byte swizzle for W2, 64-byte
 //              for W4, none for W3's 48-byte rows, so the decoders'
 //              row-per-thread 16-byte reads are bank-conflict free), and the
 //              activation tile as 64-column boxes with the 128-byte swizzle.
-//   warp 5     TMEM owner and MMA issuer: tcgen05.mma kind::f16 with A from
+//   warp 9     TMEM owner and MMA issuer: tcgen05.mma kind::f16 with A from
 //              TMEM (decoded weights) and B from shared memory
 //              (activations), FP32 accumulators in TMEM, double-buffered so
 //              the next tile's MMAs overlap the previous tile's epilogue.
-//   warps 6-9  epilogue: tcgen05.ld of the accumulator, output conversion,
+//   warps 10-13 epilogue: tcgen05.ld of the accumulator, output conversion,
 //              SwiGLU, stream-K partials and their reduction.
 //
 // This follows the article's fused A16 path ("压缩权重必须“边解码、边计算”"):
@@ -44,13 +45,15 @@ namespace cq {
 
 constexpr int kRows = 128;            // weight rows per tile (MMA M)
 constexpr int kSlice = 128;           // codes per slice along K
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr int kTmemCols = 512;
 constexpr int kTmemRing = 4;          // TMEM slice buffers (64 columns each)
 constexpr int kDCol = 256;            // first TMEM column of the accumulators
-constexpr int kDecoders = 128;
+constexpr int kDecoders = 256;        // two threads per weight row
 constexpr int kEpilogue = 128;
-constexpr int kEpiWarp0 = 6;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kEpiWarp0 = 10;
 
 template <int NT>
 struct EngineCfg {
@@ -141,10 +144,16 @@ struct EngineParams {
       prof_t = now_;                                                        \
     }                                                                       \
   } while (0)
+#define PROF_COUNT(k)                                                       \
+  do {                                                                      \
+    if (p.trace) prof[(k)] += 1;                                            \
+  } while (0)
 #define PROF_FLUSH(base)                                                    \
   do {                                                                      \
-    if (p.trace)                                                            \
-      for (int k_ = 0; k_ < 8; ++k_) p.trace[blockIdx.x * 64 + (base) + k_] = prof[k_]; \
+    if (p.trace) {                                                          \
+      _Pragma("unroll") for (int k_ = 0; k_ < 8; ++k_)                      \
+        p.trace[blockIdx.x * 64 + (base) + k_] = prof[k_];                  \
+    }                                                                       \
   } while (0)
 
 // Load through a pointer that is null in plain mode.  The volatile asm can
@@ -260,8 +269,8 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
 // with L_u = BF16(FP32(s sign(k) q(t))) the level of code u.  Levels are odd
 // in k (q(t) carries the sign), so only the positive side is evaluated in
 // FP64 and the negative codes flip the BF16 sign bit.
-template <int B>
-__device__ __forceinline__ void build_table(uint32_t tbl, uint32_t tid4, bool valid, float s,
+template <int B, int HALF>
+__device__ __forceinline__ void build_table(uint32_t* tbl, int i, bool valid, float s,
                                             uint32_t abw, int mode) {
   constexpr int H = 1 << (B - 1);
   uint32_t L[1 << B];
@@ -289,70 +298,85 @@ __device__ __forceinline__ void build_table(uint32_t tbl, uint32_t tid4, bool va
 #pragma unroll
     for (int u = 0; u < (1 << B); ++u) L[u] = 0u;
   }
+  // this thread writes entries [half * E/2, (half + 1) * E/2)
   if constexpr (B == 2) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) sts32(tbl + (e << 9) + tid4, L[e & 3] | (L[e >> 2] << 16));
+    for (int k = 0; k < 8; ++k) {
+      const int e = HALF * 8 + k;
+      tbl[e * kRows + i] = L[e & 3] | (L[e >> 2] << 16);
+    }
   } else if constexpr (B == 3) {
 #pragma unroll
-    for (int e = 0; e < 64; ++e) sts32(tbl + (e << 9) + tid4, L[e & 7] | (L[e >> 3] << 16));
+    for (int k = 0; k < 32; ++k) {
+      const int e = HALF * 32 + k;
+      tbl[e * kRows + i] = L[e & 7] | (L[e >> 3] << 16);
+    }
   } else {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) sts32(tbl + (e << 9) + tid4, L[e] | (L[e] << 16));
+    for (int k = 0; k < 8; ++k) {
+      const int e = HALF * 8 + k;
+      tbl[e * kRows + i] = L[e] | (L[e] << 16);
+    }
   }
 }
 
-// Bits [sh, sh+6) of word w moved to bit 9 (the table's entry stride).
-__device__ __forceinline__ uint32_t at_bit9(uint32_t w, int sh) {
-  return sh >= 9 ? (w >> (sh - 9)) : (w << (9 - sh));
+// Bits [sh, ...) of word w moved to bit 7 (the table's entry stride in words).
+__device__ __forceinline__ uint32_t at_bit7(uint32_t w, int sh) {
+  return sh >= 7 ? (w >> (sh - 7)) : (w << (7 - sh));
 }
 
 // Decode pairs [P0, P0+32) of one 128-code slice (codes in c[]) into r[].
 template <int B, int P0>
-__device__ __forceinline__ void decode_half(const uint32_t (&c)[4 * B], uint32_t tbl,
-                                            uint32_t tid4, uint32_t (&r)[32]) {
+__device__ __forceinline__ void decode_half(const uint32_t (&c)[4 * B], const uint32_t* tbl,
+                                            uint32_t i, uint32_t (&r)[32]) {
 #pragma unroll
   for (int q = 0; q < 32; ++q) {
     const int p = P0 + q;
     if constexpr (B == 2) {
-      const uint32_t v = at_bit9(c[p >> 3], 4 * (p & 7));
-      r[q] = lds32(tbl + ((v & (15u << 9)) | tid4));
+      const uint32_t v = at_bit7(c[p >> 3], 4 * (p & 7));
+      r[q] = tbl[(v & (15u << 7)) | i];
     } else if constexpr (B == 3) {
       const int o = 6 * p;
       const int wi = o >> 5, sh = o & 31;
       uint32_t v;
       if (sh <= 26)
-        v = at_bit9(c[wi], sh);
+        v = at_bit7(c[wi], sh);
       else
-        v = __funnelshift_r(c[wi], c[wi + 1 < 4 * B ? wi + 1 : 4 * B - 1], sh - 9);
-      r[q] = lds32(tbl + ((v & (63u << 9)) | tid4));
+        v = __funnelshift_r(c[wi], c[wi + 1 < 4 * B ? wi + 1 : 4 * B - 1], sh - 7);
+      r[q] = tbl[(v & (63u << 7)) | i];
     } else {
       const int sh = 8 * (p & 3);
       const uint32_t w = c[p >> 2];
-      const uint32_t lo = lds32(tbl + ((at_bit9(w, sh) & (15u << 9)) | tid4));
-      const uint32_t hi = lds32(tbl + ((at_bit9(w, sh + 4) & (15u << 9)) | tid4));
+      const uint32_t lo = tbl[(at_bit7(w, sh) & (15u << 7)) | i];
+      const uint32_t hi = tbl[(at_bit7(w, sh + 4) & (15u << 7)) | i];
       r[q] = __byte_perm(lo, hi, 0x7610);
     }
   }
 }
 
-template <int B>
-__device__ __forceinline__ void decode_slice_to_tmem(uint32_t codes_addr, uint32_t swz,
-                                                     uint32_t tbl, uint32_t tid4,
-                                                     uint32_t taddr) {
+// Decode pairs [32*HALF, 32*HALF+32) of one slice into TMEM columns
+// taddr .. taddr+31 (taddr already offset by 32*HALF).
+template <int B, int HALF>
+__device__ __forceinline__ void decode_half_slice_to_tmem(const uint4* codes, uint32_t swz,
+                                                          const uint32_t* tbl, uint32_t i,
+                                                          uint32_t taddr) {
   uint32_t c[4 * B];
 #pragma unroll
   for (int v = 0; v < B; ++v) {
-    const uint4 q = lds128(codes_addr + 16 * (v ^ swz));
-    c[4 * v + 0] = q.x;
-    c[4 * v + 1] = q.y;
-    c[4 * v + 2] = q.z;
-    c[4 * v + 3] = q.w;
+    // only the 16-byte chunks holding this half's bits are needed
+    if ((v + 1) * 128 > HALF * 32 * 2 * B && v * 128 < (HALF + 1) * 32 * 2 * B) {
+      const uint4 q = codes[v ^ swz];
+      c[4 * v + 0] = q.x;
+      c[4 * v + 1] = q.y;
+      c[4 * v + 2] = q.z;
+      c[4 * v + 3] = q.w;
+    } else {
+      c[4 * v + 0] = c[4 * v + 1] = c[4 * v + 2] = c[4 * v + 3] = 0u;
+    }
   }
   uint32_t r[32];
-  decode_half<B, 0>(c, tbl, tid4, r);
+  decode_half<B, 32 * HALF>(c, tbl, i, r);
   tmem_st32(taddr, r);
-  decode_half<B, 32>(c, tbl, tid4, r);
-  tmem_st32(taddr + 32, r);
 }
 
 // ---------------------------------------------------------------------------
@@ -449,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t misc = xchg_s + C::XCHG_BYTES;
   uint8_t* const gbase = smem_raw + (base - raw);
   float* const xchg = reinterpret_cast<float*>(gbase + (xchg_s - base));
-  const uint32_t tbl = smem_u32(s_tbl);
+  uint32_t* const tbl = s_tbl;
   // barriers and flags
   const uint32_t bar_full = misc;                         // [S]
   const uint32_t bar_wempty = bar_full + 8 * C::S;        // [S]
@@ -458,7 +482,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_dfull = bar_tfree + 8 * kTmemRing;   // [2]
   const uint32_t bar_dfree = bar_dfull + 16;              // [2]
   const uint32_t bar_fin = bar_dfree + 16;
-  const uint32_t slot_tmem = bar_fin + 8;
+  const uint32_t bar_tdone = bar_fin + 8;                 // [4] per lane quarter
+  const uint32_t bar_tready = bar_tdone + 32;             // [4]
+  const uint32_t slot_tmem = bar_tready + 32;
   volatile int* const abort_flag =
       reinterpret_cast<volatile int*>(gbase + (slot_tmem + 8 - base));
   volatile int* const last_flag =
@@ -486,16 +512,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_dfree + 8 * s, kEpilogue);
     }
     mbar_init(bar_fin, 1);
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(bar_tdone + 8 * s, 64);
+      mbar_init(bar_tready + 8 * s, 64);
+    }
     *abort_flag = 0;
     *last_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(slot_tmem, kTmemCols);
     tmem_relinquish();
     tc_fence_before();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tensormap(&xmap);
     if (!p.grouped) prefetch_tensormap(&wmap);
   }
@@ -514,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t r1 = cta < Pe ? range_begin(W, Pe, cta + 1) : W;
   const uint64_t tmo = p.timeout_ns;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     int st = 0;
     uint32_t round = 0;
@@ -563,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         PROF_ADD(1);
-        prof[2] += 1;
+        PROF_COUNT(2);
         ++load_no;
         if (++st == C::S) {
           st = 0;
@@ -587,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(bar_full + 8 * s, rd & 1u, &dummy, tmo, SITE_TEARDOWN);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kRows, NT);
@@ -637,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mma_commit(bar_tfree + 8 * ts);
             PROF_ADD(3);
-            prof[4] += 1;
+            PROF_COUNT(4);
             if (++ts == kTmemRing) {
               ts = 0;
               ++tround;
@@ -662,11 +692,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(bar_fin, 0, &dummy, tmo, SITE_TEARDOWN);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ decoders
-    const int i = tid;                                   // tile row / TMEM lane
+    const int q = warp & 3;                              // TMEM lane quarter
+    const int half = warp >> 2;                          // which half of each slice
+    const int i = q * 32 + lane;                         // tile row / TMEM lane
     const uint32_t tid4 = 4u * i;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    uint32_t tgen = 0;                                   // table generations built
     int st = 0, ts = 0;
     uint32_t round = 0, tround = 0;
     bool ok = true;
@@ -711,13 +744,35 @@ __global__ void __launch_bounds__(kThreads, 1)
               s_next = __ldg(ti.mat.scales + static_cast<int64_t>(grow) * ng + g_next);
               ab_next = __ldg(ti.mat.ab + static_cast<int64_t>(grow) * ng + g_next);
             }
-            if (Bw == 2)
-              build_table<2>(tbl, tid4, valid, s_cur, ab_cur, p.mode);
-            else if (Bw == 3)
-              build_table<3>(tbl, tid4, valid, s_cur, ab_cur, p.mode);
-            else
-              build_table<4>(tbl, tid4, valid, s_cur, ab_cur, p.mode);
-            prof[7] += 1;
+            // both threads of the row are done with the old table ...
+            mbar_arrive(bar_tdone + 8 * q);
+            if (!wait_phase(bar_tdone + 8 * q, tgen & 1u, abort_flag, tmo, SITE_TABLE)) {
+              ok = false;
+              break;
+            }
+            if (half == 0) {
+              if (Bw == 2)
+                build_table<2, 0>(tbl, i, valid, s_cur, ab_cur, p.mode);
+              else if (Bw == 3)
+                build_table<3, 0>(tbl, i, valid, s_cur, ab_cur, p.mode);
+              else
+                build_table<4, 0>(tbl, i, valid, s_cur, ab_cur, p.mode);
+            } else {
+              if (Bw == 2)
+                build_table<2, 1>(tbl, i, valid, s_cur, ab_cur, p.mode);
+              else if (Bw == 3)
+                build_table<3, 1>(tbl, i, valid, s_cur, ab_cur, p.mode);
+              else
+                build_table<4, 1>(tbl, i, valid, s_cur, ab_cur, p.mode);
+            }
+            // ... and both halves of the new one are written
+            mbar_arrive(bar_tready + 8 * q);
+            if (!wait_phase(bar_tready + 8 * q, tgen & 1u, abort_flag, tmo, SITE_TABLE)) {
+              ok = false;
+              break;
+            }
+            ++tgen;
+            PROF_COUNT(7);
           }
           PROF_ADD(1);
           if (!wait_phase(bar_tfree + 8 * ts, (tround & 1u) ^ 1u, abort_flag, tmo,
@@ -727,20 +782,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           PROF_ADD(2);
           tc_fence_after();
-          const uint32_t taddr = tmem_base + lane_off + ts * 64;
-          const uint32_t caddr = wrow + j * C::SLICE_W_BYTES;
-          if (Bw == 2)
-            decode_slice_to_tmem<2>(caddr, swz, tbl, tid4, taddr);
-          else if (Bw == 3)
-            decode_slice_to_tmem<3>(caddr, swz, tbl, tid4, taddr);
-          else
-            decode_slice_to_tmem<4>(caddr, swz, tbl, tid4, taddr);
+          const uint32_t taddr = tmem_base + lane_off + ts * 64 + 32 * half;
+          const uint4* caddr =
+              reinterpret_cast<const uint4*>(gbase + (wrow + j * C::SLICE_W_BYTES - base));
+          if (half == 0) {
+            if (Bw == 2)
+              decode_half_slice_to_tmem<2, 0>(caddr, swz, tbl, i, taddr);
+            else if (Bw == 3)
+              decode_half_slice_to_tmem<3, 0>(caddr, swz, tbl, i, taddr);
+            else
+              decode_half_slice_to_tmem<4, 0>(caddr, swz, tbl, i, taddr);
+          } else {
+            if (Bw == 2)
+              decode_half_slice_to_tmem<2, 1>(caddr, swz, tbl, i, taddr);
+            else if (Bw == 3)
+              decode_half_slice_to_tmem<3, 1>(caddr, swz, tbl, i, taddr);
+            else
+              decode_half_slice_to_tmem<4, 1>(caddr, swz, tbl, i, taddr);
+          }
           PROF_ADD(3);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(bar_aready + 8 * ts);
           PROF_ADD(4);
-          prof[6] += 1;
+          PROF_COUNT(6);
           if (++ts == kTmemRing) {
             ts = 0;
             ++tround;
@@ -755,8 +820,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       x = sg.end;
     }
-    if (i == 0) PROF_FLUSH(24);
-    if (i == 127) PROF_FLUSH(32);
+    if (tid == 0) PROF_FLUSH(24);
+    if (tid == 255) PROF_FLUSH(32);
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                              // TMEM lane quarter
@@ -846,7 +911,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_bar_epilogue();
       }
       PROF_ADD(1);
-      prof[2] += 1;
+      PROF_COUNT(2);
       ++seg;
       x = sg.end;
     }
@@ -855,7 +920,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   __syncthreads();
   if (tid == 0 && p.trace) p.trace[blockIdx.x * 64 + 1] = clock64() - prof_start;
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
