@@ -53,14 +53,15 @@ extern "C" int cq_gemm_noalloc(const uint16_t* x, int64_t M, const uint8_t* pack
   if (sms <= 0) return CQ_ERR_CUDA;
   if (K % kSlice != 0) return CQ_ERR_UNSUPPORTED;
   if (epilogue == CQ_EPI_SWIGLU && N % kRows != 0) return CQ_ERR_UNSUPPORTED;
-  const GemmPlan g = plan_gemm(M, N, K, epilogue, sms);
-  if (g.ws_counter_bytes + g.ws_partial_bytes > kFixedScratchBytes) return CQ_ERR_WORKSPACE;
+  size_t counter_bytes = 0, total = 0;
+  gemm_scratch(M, N, K, B, G, epilogue, sms, &counter_bytes, &total);
+  if (total > kFixedScratchBytes) return CQ_ERR_WORKSPACE;
   void* scratch = nullptr;
   st = fixed_scratch_address(&scratch);
   if (st != CQ_OK) return st;
   // The array keeps the previous call's contents: the tile counters must
   // start at zero, the partial tiles are always written before being read.
-  if (cudaMemsetAsync(scratch, 0, g.ws_counter_bytes, static_cast<cudaStream_t>(stream)) !=
+  if (cudaMemsetAsync(scratch, 0, counter_bytes, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return CQ_ERR_CUDA;
   return gemm_impl(x, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype, y,

@@ -146,6 +146,64 @@ def test_gemm_small(cq, M, N, K, B, G, mode, epi, dt):
         check_gemm(y, ref, tol_b, "gemm")
     else:
         check_swiglu(y, yr, bd, dt)
+    assert cq.device_error() == (0, 0)
+
+
+# Decode-sized shapes (M <= 2 runs the GEMV kernel): every B, group sizes
+# below, at and above one 512-code quad step, ragged N, N = 1, one group per
+# row (quads that span four row blocks), SwiGLU and BF16 output.
+GEMV_CASES = [
+    # M, N,    K,    B, G,    mode, epi, dtype
+    (1, 16,   128,  2, 128,  0, 0, 0),
+    (1, 1,    512,  3, 512,  0, 0, 0),
+    (2, 37,   1024, 3, 512,  0, 0, 0),
+    (1, 300,  3072, 3, 512,  0, 0, 1),
+    (2, 512,  2048, 4, 256,  1, 0, 0),
+    (1, 256,  7168, 2, 512,  0, 1, 0),
+    (2, 384,  1024, 2, 1024, 0, 1, 1),
+    (1, 2048, 512,  4, 128,  1, 0, 0),
+    (2, 4096, 256,  3, 256,  0, 0, 0),
+]
+
+
+@pytest.mark.parametrize("M,N,K,B,G,mode,epi,dt", GEMV_CASES)
+def test_gemv_small(cq, M, N, K, B, G, mode, epi, dt):
+    test_gemm_small(cq, M, N, K, B, G, mode, epi, dt)
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_gemv_is_deterministic_and_cleans_workspace(cq, M):
+    N, K, B, G = 7168, 3072, 3, 512
+    codes, s, ab = make_matrix(("gv_det", M), N, K, B, G)
+    pk, sd, abd = to_dev(codes, s, ab, B, cq)
+    x = synthetic.activations(13, M, K).cuda()
+    ws = cq.gemm_workspace(M, N, K, B, G)
+    y1 = cq.cq_gemm(x, pk, sd, abd, N, K, B, G, workspace=ws)
+    y2 = cq.cq_gemm(x, pk, sd, abd, N, K, B, G, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert int(ws[:256].view(torch.int32).abs().sum()) == 0
+    assert cq.device_error() == (0, 0)
+
+
+@pytest.mark.parametrize("M,B,epi", [(1, 3, 0), (2, 2, 0), (1, 4, 0), (2, 3, 1)])
+def test_gemv_matches_decoded_bf16_matmul(cq, M, B, epi):
+    """Decode-sized GEMM = matmul of cq_decode's BF16 output up to FP32
+    summation order (the operand is exactly that BF16 value)."""
+    N, K, G = 1024, 3072, 512
+    codes, s, ab = make_matrix(("gv_bf16mm", M, B), N, K, B, G)
+    pk, sd, abd = to_dev(codes, s, ab, B, cq)
+    x = synthetic.activations(17 + M, M, K).cuda()
+    w = cq.cq_decode(pk, sd, abd, K, B, G, 0, cq.BF16).double()
+    ref = x.double() @ w.T
+    bound = x.double().abs() @ w.abs().T
+    y = cq.cq_gemm(x, pk, sd, abd, N, K, B, G, epilogue=0).double()
+    assert torch.all((y - ref).abs() <= 1e-5 * bound + 1e-7)
+    if epi:
+        h = cq.cq_gemm(x, pk, sd, abd, N, K, B, G, epilogue=cq.EPI_SWIGLU).double()
+        g, u = ref[:, : N // 2], ref[:, N // 2:]
+        href = g / (1 + torch.exp(-g)) * u
+        assert torch.allclose(h, href, rtol=1e-4, atol=1e-5)
 
 
 def check_swiglu(y_gpu, yr, bd, dt):
