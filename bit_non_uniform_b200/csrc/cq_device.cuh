@@ -176,47 +176,6 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// 5-D tiled tensor copy global -> shared (no multicast).
-__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, int32_t c0,
-                                            int32_t c1, int32_t c2, int32_t c3, int32_t c4,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
-      "[%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
-      "r"(bar)
-      : "memory");
-}
-
-// 5-D tiled prefetch of one box into L2 (no shared-memory destination).
-__device__ __forceinline__ void tma_prefetch_l2_5d(const CUtensorMap* map, int32_t c0,
-                                                   int32_t c1, int32_t c2, int32_t c3,
-                                                   int32_t c4) {
-  asm volatile(
-      "cp.async.bulk.prefetch.tensor.5d.L2.global.tile [%0, {%1, %2, %3, %4, %5}];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
-      : "memory");
-}
-
-// Atomic add at GPU scope with acquire-release semantics: publishes this
-// thread's (and, after a warp barrier, its warp's) earlier writes and sees
-// the writes published by earlier adders.
-__device__ __forceinline__ int atomic_add_acq_rel_gpu(int* ptr, int v) {
-  int old;
-  asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
-  return old;
-}
-
-// 2-D tiled prefetch of one box into L2 (no shared-memory destination).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t c0, int32_t c1) {
-  asm volatile(
-      "cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(c0), "r"(c1)
-      : "memory");
-}
-
 // Programmatic dependent launch: let the next kernel on the stream be
 // scheduled now / wait until the preceding kernel has completed and its
 // memory is visible.  Both are no-ops for a launch without the attribute.

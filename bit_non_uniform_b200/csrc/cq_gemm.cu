@@ -43,60 +43,48 @@ static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int epilogue, int sms
 // ---------------------------------------------------------------------------
 struct GvPlan {
   bool use;
-  int MT, ng, spc, gpair, n_rb, n_cols, n_tasks, P, x_bytes, smem, max_quads, max_tasks;
-  size_t ws_counter_bytes, ws_partial_bytes;
+  int MT, ng, spc, gpair, n_rb, n_cols, rpc, P, x_bytes, smem, max_quads;
+  size_t ws_counter_bytes, ws_partial_bytes;   // zero: the GEMV needs no workspace
 };
 
-static int gv_dynamic_smem(int B, int MT, int G, int x_bytes, int mq, int mt) {
+static int gv_dynamic_smem(int B, int MT, int G, int spc, int x_bytes, int mq) {
   if (MT == 1) {
-    if (B == 2) return GvCfg<2, 1>::smem_bytes(G, x_bytes, mq, mt);
-    if (B == 3) return GvCfg<3, 1>::smem_bytes(G, x_bytes, mq, mt);
-    return GvCfg<4, 1>::smem_bytes(G, x_bytes, mq, mt);
+    if (B == 2) return GvCfg<2, 1>::smem_bytes(G, spc, x_bytes, mq);
+    if (B == 3) return GvCfg<3, 1>::smem_bytes(G, spc, x_bytes, mq);
+    return GvCfg<4, 1>::smem_bytes(G, spc, x_bytes, mq);
   }
-  if (B == 2) return GvCfg<2, 2>::smem_bytes(G, x_bytes, mq, mt);
-  if (B == 3) return GvCfg<3, 2>::smem_bytes(G, x_bytes, mq, mt);
-  return GvCfg<4, 2>::smem_bytes(G, x_bytes, mq, mt);
+  if (B == 2) return GvCfg<2, 2>::smem_bytes(G, spc, x_bytes, mq);
+  if (B == 3) return GvCfg<3, 2>::smem_bytes(G, spc, x_bytes, mq);
+  return GvCfg<4, 2>::smem_bytes(G, spc, x_bytes, mq);
 }
 
 static GvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int B, int G, int epilogue, int sms) {
   GvPlan v = {};
   if (M < 1 || M > 2 || N < 1 || K < G || B < 2 || B > 4) return v;
   if (epilogue == CQ_EPI_SWIGLU && N % 16 != 0) return v;
-  if (G / 8 * B > 256 || N >= (1 << 24)) return v;      // a group row must fit one TMA box row
+  if (G / 8 * B > 256 || N >= (1 << 24) || K >= (1 << 24)) return v;   // a group row = one box row
   v.MT = M == 1 ? 1 : 2;
   v.ng = static_cast<int>(K / G);
   v.spc = G / 128;
   v.gpair = v.ng % 2 == 0 ? 2 : 1;
   v.n_rb = static_cast<int>(epilogue == CQ_EPI_SWIGLU ? N / 16 : (N + 15) / 16);
   const int64_t n_cols = static_cast<int64_t>(v.n_rb) * v.ng;
-  const int64_t n_tasks = (n_cols + 3) / 4 * v.spc;
-  if (n_tasks >= (1 << 26)) return v;
+  if (n_cols >= (1 << 26)) return v;
   v.n_cols = static_cast<int>(n_cols);
-  v.n_tasks = static_cast<int>(n_tasks);
-  v.P = static_cast<int>(n_tasks < sms ? n_tasks : sms);
-  // per-CTA shared-memory layout: the largest quad and task counts of any CTA
+  // every CTA owns whole row blocks
+  v.rpc = (v.n_rb + sms - 1) / sms;
+  v.P = (v.n_rb + v.rpc - 1) / v.rpc;
+  if (v.rpc > kGvMaxRb) return v;
   for (int c = 0; c < v.P; ++c) {
-    const int T0 = static_cast<int>(static_cast<int64_t>(c) * n_tasks / v.P);
-    const int T1 = static_cast<int>(static_cast<int64_t>(c + 1) * n_tasks / v.P);
-    const int q0 = T0 / v.spc, q1 = (T1 - 1) / v.spc;
-    const int rb0 = 4 * q0 / v.ng;
-    const int rb1 = static_cast<int>((4 * static_cast<int64_t>(q1) + 3 < n_cols - 1
-                                          ? 4 * static_cast<int64_t>(q1) + 3
-                                          : n_cols - 1) / v.ng);
-    if (q1 - q0 + 1 > v.max_quads) v.max_quads = q1 - q0 + 1;
-    if (T1 - T0 > v.max_tasks) v.max_tasks = T1 - T0;
-    if (rb1 - rb0 + 1 > kGvMaxRb) return v;
-    // phase D's per-(output, group) sums reuse the code area
-    if (static_cast<int64_t>(rb1 - rb0 + 1) * 16 * v.MT * v.ng * 4 >
-        static_cast<int64_t>(q1 - q0 + 1) * 64 * (G / 8 * B))
-      return v;
+    const int rb0 = c * v.rpc;
+    const int rb1 = rb0 + v.rpc < v.n_rb ? rb0 + v.rpc : v.n_rb;
+    const int nq = ((rb1 * v.ng - 1) >> 2) - ((rb0 * v.ng) >> 2) + 1;
+    if (nq > v.max_quads) v.max_quads = nq;
   }
   if (v.max_quads > kGvMaxQuads) return v;
   v.x_bytes = static_cast<int>((M * K * 2 + 127) / 128 * 128);
-  v.smem = gv_dynamic_smem(B, v.MT, G, v.x_bytes, v.max_quads, v.max_tasks);
+  v.smem = gv_dynamic_smem(B, v.MT, G, v.spc, v.x_bytes, v.max_quads);
   if (v.smem > 227 * 1024) return v;
-  v.ws_counter_bytes = ((static_cast<size_t>(v.n_rb) * sizeof(int) + 255) / 256) * 256;
-  v.ws_partial_bytes = static_cast<size_t>(v.P) * kGvMaxRb * 16 * v.MT * sizeof(float);
   v.use = true;
   return v;
 }
@@ -154,8 +142,8 @@ static int encode_packed_gemv(CUtensorMap* map, const void* base, int64_t N, int
 
 static int run_gemv(const GvPlan& v, const uint16_t* x, int64_t M, const uint8_t* packed,
                     const float* scales, const uint16_t* ab, int64_t N, int64_t K, int B, int G,
-                    int grid_mode, int epilogue, int out_dtype, void* y, void* workspace,
-                    cudaStream_t stream, uint64_t timeout_ns, uint64_t* trace) {
+                    int grid_mode, int epilogue, int out_dtype, void* y, cudaStream_t stream,
+                    uint64_t timeout_ns, uint64_t* trace) {
   CUtensorMap wmap;
   int st = encode_packed_gemv(&wmap, packed, N, K, B, G, epilogue, v.gpair);
   if (st != CQ_OK) return st;
@@ -171,24 +159,17 @@ static int run_gemv(const GvPlan& v, const uint16_t* x, int64_t M, const uint8_t
   p.n_rb = v.n_rb;
   p.n_cols = v.n_cols;
   p.spc = v.spc;
-  p.n_tasks = v.n_tasks;
+  p.rpc = v.rpc;
   p.P = v.P;
   p.gpair = v.gpair;
   p.spc_magic = v.spc > 1 ? static_cast<uint32_t>(((1ull << 32) + v.spc - 1) / v.spc) : 0u;
   p.max_quads = v.max_quads;
-  p.max_tasks = v.max_tasks;
-  p.packed = packed;
-  p.row_bytes = K * B / 8;
   p.scales = scales;
   p.ab = reinterpret_cast<const uint32_t*>(ab);
   p.x = x;
   p.x_bytes = v.x_bytes;
   p.y = y;
   p.ldy = epilogue == CQ_EPI_SWIGLU ? N / 2 : N;
-  p.counter = reinterpret_cast<int*>(workspace);
-  p.counter_len = v.n_rb;
-  p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + v.ws_counter_bytes);
-  p.partial_len = static_cast<int64_t>(v.ws_partial_bytes / sizeof(float));
   p.timeout_ns = timeout_ns;
   p.trace = reinterpret_cast<unsigned long long*>(trace);
   if (v.MT == 1) {
@@ -252,13 +233,9 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
   const int sms = num_sms();
   if (sms <= 0) return CQ_ERR_CUDA;
   const GvPlan v = debug_skip ? GvPlan{} : plan_gemv(M, N, K, B, G, epilogue, sms);
-  if (v.use) {
-    const size_t need = v.ws_counter_bytes + v.ws_partial_bytes;
-    if (ws_bytes < need || !workspace) return CQ_ERR_WORKSPACE;
-    if (!aligned(workspace, 16)) return CQ_ERR_UNSUPPORTED;
+  if (v.use)
     return run_gemv(v, x, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype, y,
-                    workspace, stream, timeout_ns, trace);
-  }
+                    stream, timeout_ns, trace);
   const GemmPlan g = plan_gemm(M, N, K, epilogue, sms);
   const size_t need = g.ws_counter_bytes + g.ws_partial_bytes;
   if (ws_bytes < need || (need && !workspace)) return CQ_ERR_WORKSPACE;

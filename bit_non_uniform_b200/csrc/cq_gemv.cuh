@@ -21,22 +21,24 @@
 // only lane (c, c) feeds activations into operand column c (for two tokens,
 // lanes (2c+m, c) feed column 2c+m), so D[g][c] is exactly column c's
 // partial dot product.  Rotating the slice by c also makes the 16-byte code
-// reads conflict free.  A task is 8192 weights for every B; the CTA's share
-// of the task list is a contiguous range and its 20 warps take one task
-// each per round.
+// reads conflict free.  A task is 8192 weights for every B.
+//
+// Each CTA owns whole row blocks (ceil(row blocks / SMs) of them), so no
+// result ever crosses CTAs: the launch uses fewer CTAs than SMs when the
+// row blocks do not divide evenly, and a quad that straddles two CTAs' row
+// blocks is decoded by both (each keeps its own columns).
 //
 // Phases of a CTA:
-//   A  one thread: barriers and an L2 prefetch of the CTA's weight rows (safe
-//      before the preceding kernel has finished); then every thread waits for
-//      the preceding grid (programmatic dependent launch).
-//   B  one thread issues the TMA loads (one box per pair of columns: 16 rows
-//      x whole group rows) and the activation copy; all threads build every
-//      level table of the CTA's quads (FP64 levels -> FP32 -> BF16 pairs).
-//   C  warps decode and multiply their tasks; a task's partial results go to
-//      a shared slot.
-//   D  row-block sums in a fixed order (deterministic), the SwiGLU epilogue,
-//      and for row blocks shared with a neighbouring CTA the cross-CTA
-//      reduction (the last contributor sums the partials in CTA order).
+//   A  one thread sets up the barriers; every thread waits for the
+//      preceding grid (programmatic dependent launch).
+//   B  one warp issues the TMA loads (one box per pair of columns: 16 rows x
+//      whole group rows) and the activation copy; the compute warps build
+//      every level table of the CTA's quads (FP64 levels -> FP32 -> BF16
+//      pairs).
+//   C  the compute warps decode and multiply their tasks; a task's partial
+//      results go to a shared slot.
+//   D  row-block sums in a fixed order (deterministic) and the output, with
+//      the SwiGLU epilogue.
 //
 // Follows the article's A16 path (decode in the tile, model-dtype operand,
 // FP32 accumulation; the group scale folded into the BF16 level as in the
@@ -48,12 +50,12 @@
 
 namespace cq {
 
-constexpr int kGvWarps = 20;
+constexpr int kGvCompute = 12;            // warps that build tables and decode
+constexpr int kGvTmaWarp = 12;            // issues the TMA loads
+constexpr int kGvWarps = 13;
 constexpr int kGvThreads = kGvWarps * 32;
-constexpr int kGvCompute = kGvWarps - 1;   // warps that build tables and decode
-constexpr int kGvTmaWarp = kGvWarps - 1;   // issues the TMA loads
 constexpr int kGvMaxQuads = 24;         // quads one CTA may touch
-constexpr int kGvMaxRb = 64;            // row blocks one CTA may touch
+constexpr int kGvMaxRb = 16;            // row blocks one CTA may own
 
 struct GemvParams {
   int N, K, G;
@@ -63,24 +65,17 @@ struct GemvParams {
   int n_rb;            // row blocks
   int n_cols;          // n_rb * ng
   int spc;             // 128-code slices per group, G / 128
-  int n_tasks;         // quads * spc (< 2^26, checked on the host)
-  int P;               // CTAs
+  int rpc;             // row blocks per CTA
+  int P;               // CTAs, ceil(n_rb / rpc)
   int gpair;           // columns per TMA box (2 when ng is even, else 1)
   uint32_t spc_magic;  // ceil(2^32 / spc) when spc > 1
   int max_quads;       // largest number of quads of one CTA (shared layout)
-  int max_tasks;       // largest number of tasks of one CTA
-  const uint8_t* packed;
-  int64_t row_bytes;   // K * B / 8
   const float* scales;
   const uint32_t* ab;  // (a | b << 16), fp16 bits
   const uint16_t* x;   // [M][K] bf16
   int x_bytes;         // shared bytes reserved for x (>= M*K*2, multiple of 128)
   void* y;
   int64_t ldy;
-  float* partial;      // [P * kGvMaxRb][16 * MT]
-  int* counter;        // [n_rb], zero between calls
-  int64_t partial_len; // floats in partial
-  int counter_len;
   uint64_t timeout_ns;
   unsigned long long* trace;   // optional [P][64] clock64 stamps, or null
 };
@@ -98,9 +93,9 @@ struct GvCfg {
   static constexpr int NV = 64 * MT;                   // values of one task partial
   // dynamic shared memory (the first 16 KB are alignment slack: the tables
   // start on a 16 KB boundary)
-  static int smem_bytes(int G, int x_bytes, int max_quads, int max_tasks) {
+  static int smem_bytes(int G, int spc, int x_bytes, int max_quads) {
     const int quad_bytes = 64 * (G / 8 * B);
-    return 16384 + max_quads * (SET_BYTES + quad_bytes) + x_bytes + max_tasks * NV * 4 +
+    return 16384 + max_quads * (SET_BYTES + quad_bytes) + x_bytes + max_quads * spc * NV * 4 +
            kGvMaxRb * 16 * MT * 4 + 8 * (kGvMaxQuads + 1) + 64;
   }
 };
@@ -180,6 +175,15 @@ __device__ __forceinline__ bool gv_wait(uint32_t bar, uint32_t parity, volatile 
   return mbar_wait(bar, parity, abort, timeout_ns, site);
 }
 
+// Warp-wide wait: every lane waits, then the warp reconverges (lanes leave
+// the bounded spin at different iterations; without the reconvergence the
+// code after the wait would run lane group by lane group).
+__device__ __forceinline__ bool gv_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort,
+                                             uint64_t timeout_ns, int site) {
+  const bool ok = gv_wait(bar, parity, abort, timeout_ns, site);
+  return __all_sync(0xffffffffu, ok) != 0;
+}
+
 __device__ __forceinline__ float gv_silu(float g) { return g / (1.0f + expf(-g)); }
 
 // n / spc (n < 2^26, spc <= 64).
@@ -187,18 +191,28 @@ __device__ __forceinline__ int gv_div_spc(const GemvParams& p, int n) {
   return p.spc == 1 ? n : static_cast<int>(__umulhi(static_cast<uint32_t>(n), p.spc_magic));
 }
 
-// CTA that owns task tau, and the first task of CTA c.
-__device__ __forceinline__ int gv_owner(const GemvParams& p, int tau) {
-  return static_cast<int>((static_cast<int64_t>(tau + 1) * p.P - 1) / p.n_tasks);
-}
-__device__ __forceinline__ int gv_first_task(const GemvParams& p, int c) {
-  return static_cast<int>(static_cast<int64_t>(c) * p.n_tasks / p.P);
-}
-
-// Tasks [t_lo, t_hi] are the ones that touch row block rb.
-__device__ __forceinline__ void gv_rb_tasks(const GemvParams& p, int rb, int& t_lo, int& t_hi) {
-  t_lo = ((rb * p.ng) >> 2) * p.spc;
-  t_hi = (((rb * p.ng + p.ng - 1) >> 2) + 1) * p.spc - 1;
+// Sum of one output (entry e0 of column 0, row block rb) over the row
+// block's columns (group order) and their slice steps (in order), reading
+// the task partials of the CTA (task k of the CTA = its k-th quad-slice).
+template <int NV, int MT>
+__device__ __forceinline__ float gv_rb_sum(const GemvParams& p, uint32_t slots, int rb, int e0,
+                                           int q_first) {
+  float v = 0.f;
+  int chi = rb * p.ng;
+  for (int gi = 0; gi < p.ng; ++gi, ++chi) {
+    const int kb = ((chi >> 2) - q_first) * p.spc;
+    const uint32_t src = slots + 4u * static_cast<uint32_t>((chi & 3) * (16 * MT) + e0);
+    float t[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      t[u] = u < p.spc ? __uint_as_float(lds32(src + 4u * static_cast<uint32_t>(NV * (kb + u))))
+                       : 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v += t[u];
+    for (int st = 4; st < p.spc; ++st)
+      v += __uint_as_float(lds32(src + 4u * static_cast<uint32_t>(NV * (kb + st))));
+  }
+  return v;
 }
 
 template <int B, int MT>
@@ -216,7 +230,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   const uint32_t codes0 = tbl0 + p.max_quads * C::SET_BYTES;          // [quads][4][16][RG]
   const uint32_t xs = codes0 + p.max_quads * quad_bytes;              // [M][K] bf16
   const uint32_t slots = xs + static_cast<uint32_t>(p.x_bytes);       // [tasks][NV] f32
-  const uint32_t outs = slots + p.max_tasks * C::NV * 4;              // [rb][16][MT] f32
+  const uint32_t outs = slots + p.max_quads * p.spc * C::NV * 4;      // [rb][16][MT] f32
   const uint32_t bars = outs + kGvMaxRb * 16 * MT * 4;
   const uint32_t bar_quad = bars;                                     // [kGvMaxQuads]
   const uint32_t bar_x = bar_quad + 8 * kGvMaxQuads;
@@ -231,16 +245,15 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   const int cta = blockIdx.x;
   const uint64_t tmo = p.timeout_ns;
 
-  // this CTA's task range and the quads and row blocks it touches
-  const int T0 = gv_first_task(p, cta);
-  const int T1 = gv_first_task(p, cta + 1);
-  const int n_loc = T1 - T0;
-  const int q_first = gv_div_spc(p, T0);
-  const int n_quads = gv_div_spc(p, T1 - 1) - q_first + 1;
-  const int rb_first = (4 * q_first) / p.ng;
-  const int last_col = min(4 * (q_first + n_quads - 1) + 3, p.n_cols - 1);
-  const int rb_last = last_col / p.ng;
-  const int n_rbl = rb_last - rb_first + 1;
+  // this CTA's row blocks, columns, quads and tasks (quad-slices)
+  const int rb_first = cta * p.rpc;
+  const int n_rbl = min(p.rpc, p.n_rb - rb_first);
+  const int col0 = rb_first * p.ng;
+  const int col1 = (rb_first + n_rbl) * p.ng;
+  const int q_first = col0 >> 2;
+  const int n_quads = ((col1 - 1) >> 2) - q_first + 1;
+  const int n_loc = n_quads * p.spc;
+  const int T0 = q_first * p.spc;
 
   // ------------------------------------------------------------------ phase A
   if (tid == 0) {
@@ -249,37 +262,11 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     for (int q = 0; q < kGvMaxQuads; ++q) mbar_init(bar_quad + 8 * q, 1);
     mbar_init(bar_x, 1);
     int bad = 0;
-    if (n_loc <= 0 || n_quads > p.max_quads || n_loc > p.max_tasks || n_rbl > kGvMaxRb ||
-        n_quads > kGvMaxQuads)
+    if (n_rbl <= 0 || n_quads > p.max_quads || n_rbl > kGvMaxRb || n_quads > kGvMaxQuads)
       bad = 32;
     flags[0] = bad;
     if (bad) atomicCAS(&g_device_error, 0, bad);
     fence_mbar_init();
-    if (!bad) {
-      // the CTA's weight rows (whole rows: a neighbour's share of a boundary
-      // row block is wanted in L2 by that neighbour anyway)
-      int r0[2], nr[2];
-      if (p.epilogue == CQ_EPI_SWIGLU) {
-        r0[0] = rb_first * 8;
-        r0[1] = (p.N >> 1) + rb_first * 8;
-        nr[0] = nr[1] = n_rbl * 8;
-      } else {
-        r0[0] = rb_first * 16;
-        nr[0] = min(n_rbl * 16, p.N - rb_first * 16);
-        r0[1] = 0;
-        nr[1] = 0;
-      }
-      for (int h = 0; h < 2; ++h) {
-        const int64_t off = static_cast<int64_t>(r0[h]) * p.row_bytes;
-        const int64_t len = static_cast<int64_t>(nr[h]) * p.row_bytes;
-        for (int64_t o = 0; o < len; o += 1 << 20) {
-          const uint32_t n = static_cast<uint32_t>(len - o < (1 << 20) ? len - o : (1 << 20));
-          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.packed + off + o),
-                       "r"(n)
-                       : "memory");
-        }
-      }
-    }
   }
   __syncthreads();
   griddep_wait();
@@ -297,13 +284,16 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     const int nbox = 4 / p.gpair;
     for (int qq = 0; qq < n_quads; ++qq) {
       const int Q = q_first + qq;
+      // boxes holding none of this CTA's columns are not loaded
       uint32_t bytes = 0;
-      for (int bx = 0; bx < nbox; ++bx)
-        if (4 * Q + bx * p.gpair < p.n_cols) bytes += static_cast<uint32_t>(box_bytes);
+      for (int bx = 0; bx < nbox; ++bx) {
+        const int chi = 4 * Q + bx * p.gpair;
+        if (chi + p.gpair > col0 && chi < col1) bytes += static_cast<uint32_t>(box_bytes);
+      }
       mbar_arrive_expect_tx(bar_quad + 8 * qq, bytes);
       for (int bx = 0; bx < nbox; ++bx) {
         const int chi = 4 * Q + bx * p.gpair;
-        if (chi >= p.n_cols) continue;
+        if (!(chi + p.gpair > col0 && chi < col1)) continue;
         const int rb = chi / p.ng;
         const int gi = chi - rb * p.ng;
         const int y0 = p.epilogue == CQ_EPI_SWIGLU ? rb * 8 : rb * 16;
@@ -314,12 +304,13 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     GV_STAMP(3);
   }
   if (warp == kGvTmaWarp) __syncwarp();
-  // level tables: one (quad, item, lane) table per thread and round
+  // level tables: one (quad, item, lane) table per thread and round; columns
+  // of other CTAs' row blocks get zero tables
   for (int id = tid; warp < kGvCompute && id < n_quads * 64; id += kGvCompute * 32) {
     const int qq = id >> 6, it = (id >> 5) & 1, ln = id & 31;
     const int g = ln >> 2, c = ln & 3;
     const int chi = 4 * (q_first + qq) + c;
-    bool valid = chi < p.n_cols;
+    bool valid = chi >= col0 && chi < col1;
     float s = 0.f;
     uint32_t abw = 0u;
     if (valid) {
@@ -349,25 +340,25 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   if (tid == 0) GV_STAMP(4);
 
   // ------------------------------------------------------------------ phase C
-  {
+  if (warp < kGvCompute) {
     const int g = lane >> 2, c = lane & 3;
     const bool x_role = MT == 1 ? (g == c) : ((g >> 1) == c);
     const int xm = MT == 1 ? 0 : (g & 1);
     // 16-byte chunk order of the code reads (keeps them conflict free)
     const int rot = B == 2 ? (g & 1) : (B == 4 ? 2 * (c >> 1) + (g & 1) : 0);
-    bool ok = warp < kGvCompute && gv_wait(bar_x, 0, flags, tmo, SITE_GV_X);
+    bool ok = gv_wait_warp(bar_x, 0, flags, tmo, SITE_GV_X);
     for (int k = warp; ok && k < n_loc; k += kGvCompute) {
-      const int tau = T0 + k;
-      const int Q = gv_div_spc(p, tau);
-      const int qq = Q - q_first;
-      const int sstep = tau - Q * p.spc;
-      if (!gv_wait(bar_quad + 8 * qq, 0, flags, tmo, SITE_GV_STAGE_FULL)) break;
+      const int qq = gv_div_spc(p, k);
+      const int Q = q_first + qq;
+      const int sstep = k - qq * p.spc;
+      if (!gv_wait_warp(bar_quad + 8 * qq, 0, flags, tmo, SITE_GV_STAGE_FULL)) break;
       const int chi = 4 * Q + c;
-      const bool cv = chi < p.n_cols;
+      const bool cv = chi >= col0 && chi < col1;
       int sc = sstep + c;
       while (sc >= p.spc) sc -= p.spc;
       const int gi = cv ? chi - (chi / p.ng) * p.ng : 0;
-      // the lane's two rows of slice sc of column c
+      // the lane's two rows of slice sc of column c (stale data for columns
+      // of other CTAs: their tables are zero)
       const uint32_t cb = codes0 + qq * quad_bytes + c * 16 * RG + g * RG + sc * C::SLICE_BYTES;
       uint32_t c0[4 * B], c1[4 * B];
 #pragma unroll
@@ -454,104 +445,23 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   }
 
   // ------------------------------------------------------------------ phase D
-  // out_f[rbl][r][m]: row slot r = 8 * item + g of row block rb_first + rbl,
-  // summed over the row block's columns (group order) and their slices (in
-  // slice-step order): first per (output, group) into the now free code
-  // area, then over the groups
+  // out_f[rbl][r][m]: row slot r = 8 * item + g of row block rb_first + rbl
   const int n_out = n_rbl * 16 * MT;
-  float* const colsum = reinterpret_cast<float*>(gbase + (codes0 - base));
-  for (int w = tid; w < n_out * p.ng; w += kGvThreads) {
-    const int o = w / p.ng;
-    const int gi = w - o * p.ng;
+  for (int o = tid; o < n_out; o += kGvThreads) {
     const int m = o % MT;
     const int r = (o / MT) & 15;
     const int rb = rb_first + o / (16 * MT);
-    const int chi = rb * p.ng + gi;
-    const int Q = chi >> 2, cc = chi & 3;
-    const int e = ((cc * 2 + (r >> 3)) * 8 + (r & 7)) * MT + m;
-    float v = 0.f;
-    for (int st = 0; st < p.spc; ++st) {
-      const int k = Q * p.spc + st - T0;
-      if (k >= 0 && k < n_loc) v += slot_f[k * C::NV + e];
-    }
-    colsum[w] = v;
-  }
-  __syncthreads();
-  for (int o = tid; o < n_out; o += kGvThreads) {
-    float v = 0.f;
-    for (int gi = 0; gi < p.ng; ++gi) v += colsum[o * p.ng + gi];
-    out_f[o] = v;
+    out_f[o] = gv_rb_sum<C::NV, MT>(p, slots, rb, r * MT + m, q_first);
   }
   __syncthreads();
   if (tid == 0) GV_STAMP(6);
-  // row blocks whose tasks span several CTAs: publish, count, the last
-  // contributor sums every contributor's partial in CTA order
-  volatile int* const last_of = reinterpret_cast<volatile int*>(slot_f);   // slots are free now
-  bool any_partial = false;
-  for (int rbl = 0; rbl < n_rbl; ++rbl) {
-    int t_lo, t_hi;
-    gv_rb_tasks(p, rb_first + rbl, t_lo, t_hi);
-    if (t_lo >= T0 && t_hi < T1) continue;
-    any_partial = true;
-    const int64_t pslot = static_cast<int64_t>(cta) * kGvMaxRb + rbl;
-    if ((pslot + 1) * 16 * MT > p.partial_len) {
-      if (tid == 0) atomicCAS(&g_device_error, 0, 33);
-      continue;
-    }
-    for (int o = tid; o < 16 * MT; o += kGvThreads)
-      p.partial[pslot * 16 * MT + o] = out_f[rbl * 16 * MT + o];
-  }
-  if (any_partial) {
-    __syncthreads();
-    if (tid == 0) GV_STAMP(7);
-    for (int rbl = tid; rbl < n_rbl; rbl += kGvThreads) {
-      const int rb = rb_first + rbl;
-      int t_lo, t_hi;
-      gv_rb_tasks(p, rb, t_lo, t_hi);
-      int is_last = 1;
-      if (!(t_lo >= T0 && t_hi < T1)) {
-        const int c_lo = gv_owner(p, t_lo), c_hi = gv_owner(p, t_hi);
-        is_last = (rb < p.counter_len &&
-                   atomic_add_acq_rel_gpu(p.counter + rb, 1) == c_hi - c_lo) ? 1 : 0;
-        if (is_last && rb < p.counter_len) p.counter[rb] = 0;
-      }
-      last_of[rbl] = is_last;
-    }
-    __syncthreads();
-    if (tid == 0) GV_STAMP(8);
-    for (int o = tid; o < n_out; o += kGvThreads) {
-      const int rbl = o / (16 * MT);
-      const int rb = rb_first + rbl;
-      int t_lo, t_hi;
-      gv_rb_tasks(p, rb, t_lo, t_hi);
-      if ((t_lo >= T0 && t_hi < T1) || !last_of[rbl]) continue;
-      const int c_lo = gv_owner(p, t_lo), c_hi = gv_owner(p, t_hi);
-      float v = 0.f;
-      for (int cc = c_lo; cc <= c_hi; ++cc) {
-        const int crb0 = (4 * gv_div_spc(p, gv_first_task(p, cc))) / p.ng;
-        const int64_t ps = static_cast<int64_t>(cc) * kGvMaxRb + (rb - crb0);
-        if (rb - crb0 < 0 || rb - crb0 >= kGvMaxRb || (ps + 1) * 16 * MT > p.partial_len) {
-          atomicCAS(&g_device_error, 0, 34);
-          continue;
-        }
-        v += __ldcg(p.partial + ps * 16 * MT + (o - rbl * 16 * MT));
-      }
-      out_f[o] = v;
-    }
-    __syncthreads();
-    if (tid == 0) GV_STAMP(9);
-  }
-  // outputs of the row blocks this CTA finishes
   if (p.epilogue == CQ_EPI_SWIGLU) {
     for (int o = tid; o < n_rbl * 8 * MT; o += kGvThreads) {
       const int m = o % MT;
       const int g = (o / MT) & 7;
       const int rbl = o / (8 * MT);
       const int rb = rb_first + rbl;
-      int t_lo, t_hi;
-      gv_rb_tasks(p, rb, t_lo, t_hi);
-      const bool whole = t_lo >= T0 && t_hi < T1;
-      if ((!whole && !(any_partial && last_of[rbl])) || m >= p.M) continue;
+      if (m >= p.M) continue;
       const float gate = out_f[(rbl * 16 + g) * MT + m];
       const float up = out_f[(rbl * 16 + 8 + g) * MT + m];
       const float h = gv_silu(gate) * up;
@@ -565,13 +475,9 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     for (int o = tid; o < n_out; o += kGvThreads) {
       const int m = o % MT;
       const int r = (o / MT) & 15;
-      const int rbl = o / (16 * MT);
-      const int rb = rb_first + rbl;
-      int t_lo, t_hi;
-      gv_rb_tasks(p, rb, t_lo, t_hi);
-      const bool whole = t_lo >= T0 && t_hi < T1;
+      const int rb = rb_first + o / (16 * MT);
       const int row = rb * 16 + r;
-      if ((!whole && !(any_partial && last_of[rbl])) || m >= p.M || row >= p.N) continue;
+      if (m >= p.M || row >= p.N) continue;
       const int64_t off = static_cast<int64_t>(m) * p.ldy + row;
       if (p.out_bf16)
         reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(out_f[o]);

@@ -61,8 +61,9 @@ extern "C" int cq_gemm_noalloc(const uint16_t* x, int64_t M, const uint8_t* pack
   if (st != CQ_OK) return st;
   // The array keeps the previous call's contents: the tile counters must
   // start at zero, the partial tiles are always written before being read.
-  if (cudaMemsetAsync(scratch, 0, counter_bytes, static_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
+  if (counter_bytes &&
+      cudaMemsetAsync(scratch, 0, counter_bytes, static_cast<cudaStream_t>(stream)) !=
+          cudaSuccess)
     return CQ_ERR_CUDA;
   return gemm_impl(x, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype, y,
                    scratch, kFixedScratchBytes, static_cast<cudaStream_t>(stream),
