@@ -168,6 +168,7 @@ static int run_gemv(const GvPlan& v, const uint16_t* x, int64_t M, const uint8_t
   p.ab = reinterpret_cast<const uint32_t*>(ab);
   p.x = x;
   p.x_bytes = v.x_bytes;
+  p.smem_bytes = v.smem;
   p.y = y;
   p.ldy = epilogue == CQ_EPI_SWIGLU ? N / 2 : N;
   p.timeout_ns = timeout_ns;

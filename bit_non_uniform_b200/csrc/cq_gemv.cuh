@@ -47,6 +47,7 @@
 
 #include "cq.h"
 #include "cq_device.cuh"
+#include "cq_engine.cuh"
 
 namespace cq {
 
@@ -56,6 +57,9 @@ constexpr int kGvWarps = 13;
 constexpr int kGvThreads = kGvWarps * 32;
 constexpr int kGvMaxQuads = 24;         // quads one CTA may touch
 constexpr int kGvMaxRb = 16;            // row blocks one CTA may own
+// barriers and flags: a fixed block at the end of the dynamic shared memory
+// (the same place for every work item of a persistent CTA)
+constexpr int kGvBarBytes = 8 * (kGvMaxQuads + 1) + 64;
 
 struct GemvParams {
   int N, K, G;
@@ -74,10 +78,22 @@ struct GemvParams {
   const uint32_t* ab;  // (a | b << 16), fp16 bits
   const uint16_t* x;   // [M][K] bf16
   int x_bytes;         // shared bytes reserved for x (>= M*K*2, multiple of 128)
+  int smem_bytes;      // dynamic shared memory of the launch
   void* y;
   int64_t ldy;
   uint64_t timeout_ns;
   unsigned long long* trace;   // optional [P][64] clock64 stamps, or null
+};
+
+// The share of one CTA: row blocks [rb_first, rb_first + n_rbl) of one
+// matrix, multiplied with M activation rows; output row m goes to element
+// offset y_off[m] of y.
+struct GvCta {
+  int rb_first, n_rbl, M;
+  const uint16_t* x;       // [M][K] bf16
+  const float* scales;
+  const uint32_t* ab;
+  int64_t y_off[2];
 };
 
 #define GV_STAMP(k)                                                                 \
@@ -96,7 +112,7 @@ struct GvCfg {
   static int smem_bytes(int G, int spc, int x_bytes, int max_quads) {
     const int quad_bytes = 64 * (G / 8 * B);
     return 16384 + max_quads * (SET_BYTES + quad_bytes) + x_bytes + max_quads * spc * NV * 4 +
-           kGvMaxRb * 16 * MT * 4 + 8 * (kGvMaxQuads + 1) + 64;
+           kGvMaxRb * 16 * MT * 4 + kGvBarBytes;
   }
 };
 
@@ -216,8 +232,8 @@ __device__ __forceinline__ float gv_rb_sum(const GemvParams& p, uint32_t slots, 
 }
 
 template <int B, int MT>
-__global__ void __launch_bounds__(kGvThreads, 1)
-    gemv_kernel(const __grid_constant__ GemvParams p, const __grid_constant__ CUtensorMap wmap) {
+__device__ __forceinline__ void gemv_cta(const GemvParams& p, const CUtensorMap* wmap,
+                                         const GvCta& w, int max_quads, bool reuse) {
   using C = GvCfg<B, MT>;
   constexpr int E = C::E;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -227,11 +243,11 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   const int RG = p.G / 8 * B;                  // bytes of one group of one row
   const int quad_bytes = 64 * RG;              // 4 columns x 16 rows
   const uint32_t tbl0 = base;                                          // [quads][2][E][32]
-  const uint32_t codes0 = tbl0 + p.max_quads * C::SET_BYTES;          // [quads][4][16][RG]
-  const uint32_t xs = codes0 + p.max_quads * quad_bytes;              // [M][K] bf16
+  const uint32_t codes0 = tbl0 + max_quads * C::SET_BYTES;            // [quads][4][16][RG]
+  const uint32_t xs = codes0 + max_quads * quad_bytes;                // [M][K] bf16
   const uint32_t slots = xs + static_cast<uint32_t>(p.x_bytes);       // [tasks][NV] f32
-  const uint32_t outs = slots + p.max_quads * p.spc * C::NV * 4;      // [rb][16][MT] f32
-  const uint32_t bars = outs + kGvMaxRb * 16 * MT * 4;
+  const uint32_t outs = slots + max_quads * p.spc * C::NV * 4;        // [rb][16][MT] f32
+  const uint32_t bars = raw + static_cast<uint32_t>(p.smem_bytes - kGvBarBytes);
   const uint32_t bar_quad = bars;                                     // [kGvMaxQuads]
   const uint32_t bar_x = bar_quad + 8 * kGvMaxQuads;
   volatile int* const flags = reinterpret_cast<volatile int*>(gbase + (bar_x + 8 - base));
@@ -242,12 +258,11 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int cta = blockIdx.x;
   const uint64_t tmo = p.timeout_ns;
 
   // this CTA's row blocks, columns, quads and tasks (quad-slices)
-  const int rb_first = cta * p.rpc;
-  const int n_rbl = min(p.rpc, p.n_rb - rb_first);
+  const int rb_first = w.rb_first;
+  const int n_rbl = w.n_rbl;
   const int col0 = rb_first * p.ng;
   const int col1 = (rb_first + n_rbl) * p.ng;
   const int q_first = col0 >> 2;
@@ -259,10 +274,17 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   if (tid == 0) {
     GV_STAMP(0);
     griddep_launch_dependents();
+    if (reuse) {
+      // a persistent CTA's previous item: every phase of these barriers has
+      // completed and nothing waits on them any more
+      for (int q = 0; q < kGvMaxQuads; ++q) mbar_inval(bar_quad + 8 * q);
+      mbar_inval(bar_x);
+    }
     for (int q = 0; q < kGvMaxQuads; ++q) mbar_init(bar_quad + 8 * q, 1);
     mbar_init(bar_x, 1);
     int bad = 0;
-    if (n_rbl <= 0 || n_quads > p.max_quads || n_rbl > kGvMaxRb || n_quads > kGvMaxQuads)
+    if (n_rbl <= 0 || n_quads > max_quads || n_rbl > kGvMaxRb || n_quads > kGvMaxQuads ||
+        w.M < 1 || w.M > MT)
       bad = 32;
     flags[0] = bad;
     if (bad) atomicCAS(&g_device_error, 0, bad);
@@ -275,11 +297,11 @@ __global__ void __launch_bounds__(kGvThreads, 1)
 
   // ------------------------------------------------------------------ phase B
   if (warp == kGvTmaWarp && lane == 0) {
-    prefetch_tensormap(&wmap);
-    const uint32_t xbytes = static_cast<uint32_t>(p.M) * p.K * 2u;
+    prefetch_tensormap(wmap);
+    const uint32_t xbytes = static_cast<uint32_t>(w.M) * p.K * 2u;
     mbar_arrive_expect_tx(bar_x, xbytes);
-    for (int m = 0; m < p.M; ++m)
-      bulk_g2s(xs + m * p.K * 2, p.x + static_cast<int64_t>(m) * p.K, p.K * 2u, bar_x);
+    for (int m = 0; m < w.M; ++m)
+      bulk_g2s(xs + m * p.K * 2, w.x + static_cast<int64_t>(m) * p.K, p.K * 2u, bar_x);
     const int box_bytes = p.gpair * 16 * RG;
     const int nbox = 4 / p.gpair;
     for (int qq = 0; qq < n_quads; ++qq) {
@@ -297,7 +319,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         const int rb = chi / p.ng;
         const int gi = chi - rb * p.ng;
         const int y0 = p.epilogue == CQ_EPI_SWIGLU ? rb * 8 : rb * 16;
-        tma_load_4d(codes0 + qq * quad_bytes + bx * box_bytes, &wmap, 0, y0, 0, gi,
+        tma_load_4d(codes0 + qq * quad_bytes + bx * box_bytes, wmap, 0, y0, 0, gi,
                     bar_quad + 8 * qq);
       }
     }
@@ -320,8 +342,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       valid = row < p.N;
       if (valid) {
         const int64_t mi = static_cast<int64_t>(row) * p.ng + gi;
-        s = __ldg(p.scales + mi);
-        abw = __ldg(p.ab + mi);
+        s = __ldg(w.scales + mi);
+        abw = __ldg(w.ab + mi);
       }
     }
     uint32_t L[1 << B];
@@ -382,7 +404,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       }
       const uint32_t tl0 = tbl0 + qq * C::SET_BYTES + lane * 4;
       const uint32_t tl1 = tl0 + E * 128;
-      const bool xh = x_role && cv && xm < p.M;
+      const bool xh = x_role && cv && xm < w.M;
       const uint32_t xa = xs + (static_cast<uint32_t>(xm) * p.K + gi * p.G + sc * 128) * 2u;
       float acc[4][4];
 #pragma unroll
@@ -461,11 +483,11 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       const int g = (o / MT) & 7;
       const int rbl = o / (8 * MT);
       const int rb = rb_first + rbl;
-      if (m >= p.M) continue;
+      if (m >= w.M) continue;
       const float gate = out_f[(rbl * 16 + g) * MT + m];
       const float up = out_f[(rbl * 16 + 8 + g) * MT + m];
       const float h = gv_silu(gate) * up;
-      const int64_t off = static_cast<int64_t>(m) * p.ldy + rb * 8 + g;
+      const int64_t off = w.y_off[m] + rb * 8 + g;
       if (p.out_bf16)
         reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(h);
       else
@@ -477,8 +499,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       const int r = (o / MT) & 15;
       const int rb = rb_first + o / (16 * MT);
       const int row = rb * 16 + r;
-      if (m >= p.M || row >= p.N) continue;
-      const int64_t off = static_cast<int64_t>(m) * p.ldy + row;
+      if (m >= w.M || row >= p.N) continue;
+      const int64_t off = w.y_off[m] + row;
       if (p.out_bf16)
         reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(out_f[o]);
       else
@@ -486,6 +508,132 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     }
   }
   if (tid == 0) GV_STAMP(1);
+}
+
+// cq_gemm's decode-sized path: CTA c owns row blocks [c * rpc, (c+1) * rpc).
+template <int B, int MT>
+__global__ void __launch_bounds__(kGvThreads, 1)
+    gemv_kernel(const __grid_constant__ GemvParams p, const __grid_constant__ CUtensorMap wmap) {
+  GvCta w;
+  w.rb_first = blockIdx.x * p.rpc;
+  w.n_rbl = min(p.rpc, p.n_rb - w.rb_first);
+  w.M = p.M;
+  w.x = p.x;
+  w.scales = p.scales;
+  w.ab = p.ab;
+  w.y_off[0] = 0;
+  w.y_off[1] = p.ldy;
+  gemv_cta<B, MT>(p, &wmap, w, p.max_quads, false);
+}
+
+// ---------------------------------------------------------------------------
+// Grouped (MoE) form: the decode-sized products of one MoE stage, one work
+// item per (expert, chunk of at most MT routed tokens, range of row blocks).
+// Items are ordered by bit width (all B = 2, then 3, then 4) so that items of
+// one width are uniform; a persistent CTA walks items item, item + grid, ...
+// ---------------------------------------------------------------------------
+struct GvMatrix {        // one expert matrix (device pointers)
+  const uint8_t* packed;
+  const float* scales;
+  const uint32_t* ab;
+  int B;
+  int reserved;
+};
+
+struct alignas(64) GvExpert {   // what the grouped kernel needs of one expert and stage
+  CUtensorMap map;               // the 4-D GEMV tensor map of the matrix
+  GvMatrix mat;
+};
+
+struct MoeGvParams {
+  GemvParams base;             // shape of the stage's matrices (x, scales, ab, y unused)
+  int rpc[3];                  // row blocks per item, B = 2, 3, 4
+  int max_quads[3];
+  int ipi[3];                  // items per chunk: ceil(n_rb / rpc)
+  const GvExpert* experts;     // [E] (64-byte aligned)
+  int E;
+  const int* n_chunks;         // [3] chunks of width B (device, written by the router)
+  const int* chunk_e;          // [chunks] expert of each chunk, ordered by width
+  const int* chunk_pos;        // [chunks] sorted position of its first route
+  const int* chunk_m;          // [chunks] routes in the chunk (1..MT)
+  const uint16_t* xs;          // [R][K] bf16 activations in sorted order
+  void* y;                     // output rows
+  const int* out_rows;         // sorted position -> output row, or null (identity)
+  int64_t y_rows;              // rows of y
+  int64_t R;                   // routes (rows of xs)
+};
+
+// Resolve work item `item` of a grouped stage: width, chunk and row blocks.
+struct GvItem {
+  int bi, ck, part;
+};
+__device__ __forceinline__ bool gv_item(const MoeGvParams& q, int item, int n2, int n3, int s3,
+                                        int s4, int total, GvItem& it) {
+  if (item >= total) return false;
+  int local, chunk0;
+  if (item < s3) {
+    it.bi = 0; local = item; chunk0 = 0;
+  } else if (item < s4) {
+    it.bi = 1; local = item - s3; chunk0 = n2;
+  } else {
+    it.bi = 2; local = item - s4; chunk0 = n2 + n3;
+  }
+  it.ck = chunk0 + local / q.ipi[it.bi];
+  it.part = local % q.ipi[it.bi];
+  return true;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kGvThreads, 1) moe_gemv_kernel(const __grid_constant__ MoeGvParams q) {
+  if (!q.base.y || !q.xs) {
+    if (threadIdx.x == 0) atomicCAS(&g_device_error, 0, 38);
+    return;
+  }
+  const int n2 = ld_guarded(q.n_chunks + 0), n3 = ld_guarded(q.n_chunks + 1),
+            n4 = ld_guarded(q.n_chunks + 2);
+  const int s3 = n2 * q.ipi[0];
+  const int s4 = s3 + n3 * q.ipi[1];
+  const int total = s4 + n4 * q.ipi[2];
+  bool reuse = false;
+  GvItem cur;
+  for (int item = blockIdx.x; item < total; item += gridDim.x) {
+    gv_item(q, item, n2, n3, s3, s4, total, cur);
+    const int bi = cur.bi, ck = cur.ck, part = cur.part;
+    const int e = ld_guarded(q.chunk_e + ck);
+    const int pos = ld_guarded(q.chunk_pos + ck);
+    const int M = ld_guarded(q.chunk_m + ck);
+    if (e < 0 || e >= q.E || pos < 0 || M < 1 || M > MT || pos + M > q.R) {
+      if (threadIdx.x == 0) atomicCAS(&g_device_error, 0, 36);
+      continue;
+    }
+    const GvExpert* ex = q.experts + e;
+    GvCta w;
+    w.rb_first = part * q.rpc[bi];
+    w.n_rbl = min(q.rpc[bi], q.base.n_rb - w.rb_first);
+    w.M = M;
+    w.x = q.xs + static_cast<int64_t>(pos) * q.base.K;
+    w.scales = ex->mat.scales;
+    w.ab = ex->mat.ab;
+    bool rows_ok = true;
+    for (int m = 0; m < 2; ++m) {
+      const int pm = pos + (m < M ? m : 0);
+      const int64_t row = q.out_rows ? static_cast<int64_t>(ld_guarded(q.out_rows + pm)) : pm;
+      if (row < 0 || row >= q.y_rows) rows_ok = false;
+      w.y_off[m] = row * q.base.ldy;
+    }
+    if (!rows_ok || ex->mat.B != bi + 2) {
+      if (threadIdx.x == 0) atomicCAS(&g_device_error, 0, 37);
+      continue;
+    }
+    if (bi == 0)
+      gemv_cta<2, MT>(q.base, &ex->map, w, q.max_quads[0], reuse);
+    else if (bi == 1)
+      gemv_cta<3, MT>(q.base, &ex->map, w, q.max_quads[1], reuse);
+    else
+      gemv_cta<4, MT>(q.base, &ex->map, w, q.max_quads[2], reuse);
+    reuse = true;
+    __syncthreads();
+  }
 }
 
 }  // namespace cq

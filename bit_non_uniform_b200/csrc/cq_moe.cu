@@ -7,6 +7,7 @@
 
 #include "cq.h"
 #include "cq_engine.cuh"
+#include "cq_gemv.cuh"
 #include "cq_host.h"
 
 namespace cq {
@@ -15,7 +16,10 @@ constexpr int kRouteThreads = 1024;
 constexpr int kMaxExperts = 16384;     // routing counters live in shared memory
 
 // control words at the head of the workspace
-enum Ctrl : int { CTRL_TT = 0, CTRL_TILES_GU = 1, CTRL_TILES_DN = 2, CTRL_BAD = 3 };
+enum Ctrl : int {
+  CTRL_TT = 0, CTRL_TILES_GU = 1, CTRL_TILES_DN = 2, CTRL_BAD = 3,
+  CTRL_CHUNKS = 8      // [2 stages][3 widths]: decode-path chunks per bit width
+};
 
 // Exclusive scan of v[0..n) in place with one CTA of kRouteThreads threads;
 // returns the total (to every thread).  Each thread owns a contiguous chunk.
@@ -58,7 +62,8 @@ __global__ void __launch_bounds__(kRouteThreads)
                      int n_rt_dn, int* __restrict__ ctrl, int* __restrict__ cnt,
                      int* __restrict__ off, int* __restrict__ ttpre, int* __restrict__ rank,
                      int* __restrict__ perm, int* __restrict__ pos_of,
-                     int* __restrict__ counters_gu, int* __restrict__ counters_dn) {
+                     int* __restrict__ counters_gu, int* __restrict__ counters_dn,
+                     const GvExpert* __restrict__ gvx, int* __restrict__ chunks, int max_chunks) {
   extern __shared__ int s_mem[];
   int* s_cnt = s_mem;                        // [E]
   int* s_tt = s_mem + E;                     // [E]
@@ -109,6 +114,37 @@ __global__ void __launch_bounds__(kRouteThreads)
   // stream-K tile counters of the two grouped launches start at zero
   for (int i = tid; i < n_rt_gu * tt_total; i += kRouteThreads) counters_gu[i] = 0;
   for (int i = tid; i < n_rt_dn * tt_total; i += kRouteThreads) counters_dn[i] = 0;
+  if (!gvx) return;
+  // decode path: chunks of at most two routes per expert, listed by bit width
+  // (B = 2, 3, 4) and, within a width, by expert; per stage
+  __syncthreads();
+  for (int stage = 0; stage < 2; ++stage) {
+    int* const ch_e = chunks + (stage * 3 + 0) * max_chunks;
+    int* const ch_pos = chunks + (stage * 3 + 1) * max_chunks;
+    int* const ch_m = chunks + (stage * 3 + 2) * max_chunks;
+    int base = 0;
+    for (int b = 2; b <= 4; ++b) {
+      for (int e = tid; e < E; e += kRouteThreads)
+        s_tt[e] = (gvx[stage * E + e].mat.B == b) ? (cnt[e] + 1) / 2 : 0;
+      __syncthreads();
+      const int n_b = block_exclusive_scan(s_tt, E, s_part);
+      for (int e = tid; e < E; e += kRouteThreads) {
+        if (gvx[stage * E + e].mat.B != b) continue;
+        const int c = cnt[e];
+        for (int j = 0; 2 * j < c; ++j) {
+          const int idx = base + s_tt[e] + j;
+          if (idx < max_chunks) {
+            ch_e[idx] = e;
+            ch_pos[idx] = off[e] + 2 * j;
+            ch_m[idx] = c - 2 * j < 2 ? c - 2 * j : 2;
+          }
+        }
+      }
+      if (tid == 0) ctrl[CTRL_CHUNKS + stage * 3 + (b - 2)] = n_b;
+      base += n_b;
+      __syncthreads();
+    }
+  }
 }
 
 // Copy each routed token's activation row to its expert-sorted position.
@@ -182,9 +218,9 @@ static int moe_pick_nt(int64_t R, int E) {
 
 struct MoePlan {
   int NT, n_rt_gu, n_rt_dn, P;
-  int64_t R, max_tt;
+  int64_t R, max_tt, max_chunks;
   size_t o_ctrl, o_cnt, o_off, o_ttpre, o_rank, o_perm, o_pos, o_x, o_h, o_y, o_cgu, o_cdn,
-      o_part, total;
+      o_part, o_chunks, total;
 };
 
 static MoePlan moe_plan(int64_t T, int k, int E, int64_t H, int64_t I, int sms) {
@@ -215,6 +251,9 @@ static MoePlan moe_plan(int64_t T, int k, int E, int64_t H, int64_t I, int sms) 
   m.o_cgu = take(static_cast<size_t>(m.n_rt_gu) * m.max_tt * sizeof(int));
   m.o_cdn = take(static_cast<size_t>(m.n_rt_dn) * m.max_tt * sizeof(int));
   m.o_part = take(static_cast<size_t>(2) * m.P * m.NT * kRows * sizeof(float));
+  // decode path: sum over experts of ceil(cnt/2) <= (R + active experts) / 2
+  m.max_chunks = (m.R + (m.R < E ? m.R : E)) / 2 + 1;
+  m.o_chunks = take(static_cast<size_t>(6) * m.max_chunks * sizeof(int));
   m.total = o;
   return m;
 }
@@ -226,6 +265,57 @@ static int validate_moe_shape(int64_t T, int k, int E, int64_t H, int64_t I, int
   if (T * k > (int64_t)1 << 28 || H > (int64_t)1 << 20 || I > (int64_t)1 << 20)
     return CQ_ERR_UNSUPPORTED;
   return CQ_OK;
+}
+
+// Decode-sized grouped path: usable when experts see few routes on average
+// and the GEMV kernel fits every bit width's work item in shared memory.
+static bool moe_gemv_plan(const MoePlan& m, int64_t T, int k, int E, int64_t H, int64_t I, int G,
+                          int grid_mode, int sms, MoeGvParams* q) {
+  const int64_t active = m.R < E ? m.R : E;
+  if (m.R > 4 * active || G / 8 * 4 > 256) return false;
+  for (int stage = 0; stage < 2; ++stage) {
+    const int64_t N = stage == 0 ? 2 * I : H;
+    const int64_t K = stage == 0 ? H : I;
+    MoeGvParams& p = q[stage];
+    memset(&p, 0, sizeof(p));
+    GemvParams& b = p.base;
+    b.N = static_cast<int>(N);
+    b.K = static_cast<int>(K);
+    b.G = G;
+    b.mode = grid_mode;
+    b.epilogue = stage == 0 ? CQ_EPI_SWIGLU : CQ_EPI_NONE;
+    b.out_bf16 = stage == 0 ? 1 : 0;
+    b.M = 2;
+    b.ng = static_cast<int>(K / G);
+    b.n_rb = static_cast<int>(stage == 0 ? N / 16 : (N + 15) / 16);
+    b.n_cols = b.n_rb * b.ng;
+    b.spc = G / 128;
+    b.gpair = b.ng % 2 == 0 ? 2 : 1;
+    b.spc_magic = b.spc > 1 ? static_cast<uint32_t>(((1ull << 32) + b.spc - 1) / b.spc) : 0u;
+    b.x_bytes = static_cast<int>((2 * K * 2 + 127) / 128 * 128);
+    b.ldy = stage == 0 ? I : H;
+    b.timeout_ns = kDefaultTimeoutNs;
+    int smem = 0;
+    for (int bi = 0; bi < 3; ++bi) {
+      const int B = bi + 2;
+      int rpc = (b.n_rb + sms - 1) / sms;
+      if (rpc > kGvMaxRb) rpc = kGvMaxRb;
+      int sm = 0, mq = 0;
+      for (; rpc >= 1; --rpc) {
+        mq = (rpc * b.ng + 3) / 4 + 1;
+        if (mq > kGvMaxQuads) continue;
+        sm = gv_dynamic_smem(B, 2, G, b.spc, b.x_bytes, mq);
+        if (sm <= 227 * 1024) break;
+      }
+      if (rpc < 1) return false;
+      p.rpc[bi] = rpc;
+      p.max_quads[bi] = mq;
+      p.ipi[bi] = (b.n_rb + rpc - 1) / rpc;
+      if (sm > smem) smem = sm;
+    }
+    b.smem_bytes = smem;
+  }
+  return true;
 }
 
 template <int NT>
@@ -249,8 +339,13 @@ static int launch_grouped_nt(int NT, const EngineParams& p, const CUtensorMap& x
 
 using namespace cq;
 
+// Layer table: [E] LayerEntry (engine) followed by [2][E] GvExpert (the
+// decode-sized path's per-expert tensor maps; a B whose group rows do not fit
+// one box row leaves the map zero and the layer on the engine).
+static size_t gv_table_offset(int E) { return static_cast<size_t>(E) * sizeof(LayerEntry); }
+
 extern "C" size_t cq_moe_layer_bytes(int E) {
-  return E > 0 ? static_cast<size_t>(E) * sizeof(LayerEntry) : 0;
+  return E > 0 ? gv_table_offset(E) + static_cast<size_t>(2) * E * sizeof(GvExpert) : 0;
 }
 
 extern "C" int cq_moe_prepare_layer(const cq_expert_desc* experts, int E, int64_t H, int64_t I,
@@ -261,6 +356,8 @@ extern "C" int cq_moe_prepare_layer(const cq_expert_desc* experts, int E, int64_
   if (!aligned(layer, 64)) return CQ_ERR_UNSUPPORTED;
   std::vector<LayerEntry> host(static_cast<size_t>(E));
   memset(host.data(), 0, host.size() * sizeof(LayerEntry));
+  std::vector<GvExpert> gvx(static_cast<size_t>(2) * E);
+  memset(gvx.data(), 0, gvx.size() * sizeof(GvExpert));
   for (int e = 0; e < E; ++e) {
     const cq_matrix_desc* d[2] = {&experts[e].gate_up, &experts[e].down};
     const int64_t rows[2] = {2 * I, H};
@@ -278,10 +375,24 @@ extern "C" int cq_moe_prepare_layer(const cq_expert_desc* experts, int E, int64_
       host[e].mat[w].ab = reinterpret_cast<const uint32_t*>(d[w]->ab);
       host[e].mat[w].B = d[w]->B;
       host[e].mat[w].reserved = 0;
+      GvExpert& g = gvx[static_cast<size_t>(w) * E + e];
+      g.mat.packed = d[w]->packed;
+      g.mat.scales = d[w]->scales;
+      g.mat.ab = reinterpret_cast<const uint32_t*>(d[w]->ab);
+      g.mat.B = d[w]->B;
+      if (G / 8 * d[w]->B <= 256) {
+        const int ng = static_cast<int>(cols[w] / G);
+        st = encode_packed_gemv(&g.map, d[w]->packed, rows[w], cols[w], d[w]->B, G,
+                                w == 0 ? CQ_EPI_SWIGLU : CQ_EPI_NONE, ng % 2 == 0 ? 2 : 1);
+        if (st != CQ_OK) return st;
+      }
     }
   }
   if (cudaMemcpy(layer, host.data(), host.size() * sizeof(LayerEntry),
                  cudaMemcpyHostToDevice) != cudaSuccess)
+    return CQ_ERR_CUDA;
+  if (cudaMemcpy(static_cast<uint8_t*>(layer) + gv_table_offset(E), gvx.data(),
+                 gvx.size() * sizeof(GvExpert), cudaMemcpyHostToDevice) != cudaSuccess)
     return CQ_ERR_CUDA;
   return CQ_OK;
 }
@@ -338,9 +449,15 @@ extern "C" int cq_moe_grouped_gemm(const uint16_t* tokens, int64_t T, const int3
       return CQ_ERR_CUDA;
     route_attr = true;
   }
-  moe_route_kernel<<<1, kRouteThreads, route_smem, s>>>(topk_ids, R, E, m.NT, m.n_rt_gu,
-                                                        m.n_rt_dn, ctrl, cnt, off, ttpre, rank,
-                                                        perm, pos_of, cgu, cdn);
+  // decode-sized layers (few routes per expert) take the grouped GEMV path
+  MoeGvParams gvp[2];
+  const bool gv = moe_gemv_plan(m, T, k, E, H, I, G, grid_mode, sms, gvp);
+  const GvExpert* gvx = reinterpret_cast<const GvExpert*>(
+      static_cast<const uint8_t*>(layer) + gv_table_offset(E));
+  int* chunks = reinterpret_cast<int*>(ws + m.o_chunks);
+  moe_route_kernel<<<1, kRouteThreads, route_smem, s>>>(
+      topk_ids, R, E, m.NT, m.n_rt_gu, m.n_rt_dn, ctrl, cnt, off, ttpre, rank, perm, pos_of,
+      cgu, cdn, gv ? gvx : nullptr, chunks, static_cast<int>(m.max_chunks));
   if (cudaGetLastError() != cudaSuccess) return CQ_ERR_CUDA;
   // 2. expert-sorted activations
   const int row16 = static_cast<int>(H * 2 / 16);
@@ -349,11 +466,37 @@ extern "C" int cq_moe_grouped_gemm(const uint16_t* tokens, int64_t T, const int3
   if (cudaGetLastError() != cudaSuccess) return CQ_ERR_CUDA;
   // 3. gate/up + SwiGLU -> h (BF16, sorted order);  4. down -> y (FP32, route order)
   CUtensorMap xmap_gu, xmap_dn;
+  if (gv) {
+    for (int stage = 0; stage < 2; ++stage) {
+      MoeGvParams& q = gvp[stage];
+      q.experts = gvx + static_cast<size_t>(stage) * E;
+      q.E = E;
+      q.n_chunks = ctrl + CTRL_CHUNKS + 3 * stage;
+      q.chunk_e = chunks + (stage * 3 + 0) * m.max_chunks;
+      q.chunk_pos = chunks + (stage * 3 + 1) * m.max_chunks;
+      q.chunk_m = chunks + (stage * 3 + 2) * m.max_chunks;
+      q.xs = stage == 0 ? xs : hs;
+      q.y = stage == 0 ? static_cast<void*>(hs) : static_cast<void*>(ybuf);
+      q.base.y = q.y;                  // the per-CTA body writes through the stage shape
+      q.out_rows = stage == 0 ? nullptr : perm;
+      q.y_rows = m.R;
+      q.R = m.R;
+      static bool attr = false;
+      if (!attr) {
+        if (cudaFuncSetAttribute(moe_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 227 * 1024) != cudaSuccess)
+          return CQ_ERR_CUDA;
+        attr = true;
+      }
+      moe_gemv_kernel<2><<<sms, kGvThreads, q.base.smem_bytes, s>>>(q);
+      if (cudaGetLastError() != cudaSuccess) return CQ_ERR_CUDA;
+    }
+  }
   st = encode_bf16_rows_sw128(&xmap_gu, xs, R, H, m.NT);
   if (st != CQ_OK) return st;
   st = encode_bf16_rows_sw128(&xmap_dn, hs, R, I, m.NT);
   if (st != CQ_OK) return st;
-  for (int which = 0; which < 2; ++which) {
+  for (int which = 0; which < 2 && !gv; ++which) {
     EngineParams p = {};
     p.N = static_cast<int>(which == 0 ? 2 * I : H);
     p.K = static_cast<int>(which == 0 ? H : I);

@@ -64,6 +64,10 @@ TOY = [
     (512, 256, 8, 37, 2, 128, (2, 3, 4), "uniform"),
     (512, 256, 4, 300, 2, 256, (3, 4), "uniform"),     # ~150 tokens per expert: several tiles
     (1024, 512, 16, 9, 4, 512, (2,), "zipf"),
+    # few routes per expert: the decode-sized grouped path, mixed widths,
+    # experts with one, two and more routes (chunks of two)
+    (512, 256, 32, 24, 2, 128, (2, 3, 4), "uniform"),
+    (1024, 512, 16, 24, 2, 512, (3, 4), "zipf"),
 ]
 
 
