@@ -54,6 +54,42 @@ WORKLOADS = {
 }
 
 
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture
+# (profiles/gemv_kernel_down_w3g512_m1.md).  Keyed by the SHA-256 of the kernel's
+# sources at capture time: once they change, the figure no longer describes the
+# kernel and `traffic` is reported as null.
+KERNEL_SOURCES = ("cq_gemv.cuh", "cq_gemm.cu", "cq_device.cuh", "cq_engine.cuh")
+TRAFFIC = {
+    "down_m1": {"kernel": "gemv_kernel<3,1>", "bytes": 8651776,
+                "sources_sha256": "a5eed5894780ada6febe7c8e501679bbda13e4754e7e44eb28999b674ff9c265"},
+}
+
+
+def kernel_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "bit_non_uniform_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(name):
+    rec = TRAFFIC.get(name)
+    if rec is None or rec["sources_sha256"] != kernel_sources_sha256():
+        return None
+    return rec["bytes"]
+
+
+def dominant_kernel(name):
+    """The kernel one cq_gemm launch of the workload runs (the only one it runs)."""
+    _, N, K, B, G, M, epi = WORKLOADS[name]
+    if M <= 2:
+        return f"gemv_kernel<{B},{M}>"
+    nt = 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
+    return f"engine_kernel<{nt}>"
+
+
 def packed_bytes(N, K, B, G):
     return N * K * B // 8 + N * (K // G) * 8
 
@@ -161,9 +197,17 @@ def max_over_ranks(v: float, world: int) -> float:
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, ms_per_rank: float, world: int) -> float:
+    """Whole-job throughput of replicas: every rank processes the same units,
+    the job takes as long as the slowest rank (units per ms, all ranks)."""
+    slowest = max_over_ranks(ms_per_rank, world)
+    return units_per_rank * world / slowest
 
 
 # --------------------------------------------------------------------------
@@ -516,7 +560,7 @@ def main():
     r = main_res
     value = r["gbs"] * world          # every rank streams its own replica
     ach = r["alg_bytes"] / (r["ms_per_step"] * 1e-3) / 1e9
-    traffic = None
+    traffic = measured_traffic(args.workload)
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -537,7 +581,7 @@ def main():
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(ach / hbm, 4), "traffic": traffic,
-                     "peak_source": peak_src},
+                     "kernel": dominant_kernel(args.workload), "peak_source": peak_src},
         "e2e": e2e,
         "gpu_launches": args.steps,
         "clocks": r["clocks"],
