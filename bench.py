@@ -58,7 +58,7 @@ WORKLOADS = {
 # (profiles/gemv_kernel_down_w3g512_m1.md).  Keyed by the SHA-256 of the kernel's
 # sources at capture time: once they change, the figure no longer describes the
 # kernel and `traffic` is reported as null.
-KERNEL_SOURCES = ("cq_gemv.cuh", "cq_gemm.cu", "cq_device.cuh", "cq_engine.cuh")
+KERNEL_SOURCES = ("cq_gemv.cuh", "cq_gemv_launch.cuh", "cq_device.cuh")
 TRAFFIC = {
     "down_m1": {"kernel": "gemv_kernel<3,1>", "bytes": 8651776,
                 "sources_sha256": "a5eed5894780ada6febe7c8e501679bbda13e4754e7e44eb28999b674ff9c265"},

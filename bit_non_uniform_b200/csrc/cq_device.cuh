@@ -354,6 +354,16 @@ __device__ __forceinline__ double level_f64(int u, int B, int mode, float s, dou
   return static_cast<double>(s) * static_cast<double>(sg) * q;
 }
 
+// Load through a pointer that may be null when the guarding branch is not
+// taken (plain mode of the grouped kernels).  The volatile asm can
+// neither be hoisted above the branch that guards it nor turned into an
+// unconditional load by if-conversion.
+__device__ __forceinline__ int ld_guarded(const int* ptr) {
+  int v;
+  asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(ptr));
+  return v;
+}
+
 __device__ __forceinline__ uint16_t bf16_bits(float f) {
   __nv_bfloat16 h = __float2bfloat16_rn(f);
   return *reinterpret_cast<uint16_t*>(&h);

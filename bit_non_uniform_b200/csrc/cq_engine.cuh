@@ -26,7 +26,9 @@
 //   warp 9     TMEM owner and MMA issuer: tcgen05.mma kind::f16 with A from
 //              TMEM (decoded weights) and B from shared memory
 //              (activations), FP32 accumulators in TMEM, double-buffered so
-//              the next tile's MMAs overlap the previous tile's epilogue.
+//              the next tile's MMAs overlap the previous tile's epilogue
+//              (single-buffered at NT = 256, whose 256 accumulator columns
+//              fill the TMEM beside the A ring).
 //   warps 10-13 epilogue: tcgen05.ld of the accumulator, output conversion,
 //              SwiGLU, stream-K partials and their reduction.
 //
@@ -58,6 +60,9 @@ constexpr int kEpiWarp0 = 10;
 template <int NT>
 struct EngineCfg {
   static constexpr int SPS = NT <= 32 ? 4 : (NT == 64 ? 2 : 1);   // slices per stage
+  // accumulator buffers in TMEM: two (the next tile's MMAs overlap this
+  // tile's epilogue) while they fit beside the A ring, else one
+  static constexpr int NBUF = kDCol + 2 * NT <= kTmemCols ? 2 : 1;
   static constexpr int SLICE_W_BYTES = kRows * 16 * 4;          // one slice of packed rows (B<=4)
   static constexpr int W_BYTES = SPS * SLICE_W_BYTES;
   static constexpr int X_BYTES = 256 * SPS * NT;                // 2*SPS boxes of 64 x NT bf16
@@ -71,7 +76,7 @@ struct EngineCfg {
   static constexpr int SMEM = 1024 + S * STAGE_BYTES + XCHG_BYTES + MISC_BYTES;
   static_assert(S >= 2, "not enough shared memory for two stages");
   static_assert(SMEM + TBL_BYTES <= 227 * 1024, "shared memory budget exceeded");
-  static_assert(kDCol + 2 * NT <= kTmemCols, "TMEM budget exceeded");
+  static_assert(kDCol + NBUF * NT <= kTmemCols, "TMEM budget exceeded");
 };
 
 // One quantized matrix operand.
@@ -155,15 +160,6 @@ struct EngineParams {
         p.trace[blockIdx.x * 64 + (base) + k_] = prof[k_];                  \
     }                                                                       \
   } while (0)
-
-// Load through a pointer that is null in plain mode.  The volatile asm can
-// neither be hoisted above the branch that guards it nor turned into an
-// unconditional load by if-conversion.
-__device__ __forceinline__ int ld_guarded(const int* ptr) {
-  int v;
-  asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(ptr));
-  return v;
-}
 
 // Record a failed bounds check (site >= 20) in the device error word.
 __device__ __forceinline__ void bad_access(int site) { atomicCAS(&g_device_error, 0, site); }
@@ -402,38 +398,86 @@ __device__ __forceinline__ bool vote_all_epilogue(bool ok) {
   return r != 0;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
-
 // Store 16 accumulator columns (tokens m0..m0+15 of the tile) of tile row i.
 __device__ __forceinline__ void finalize16(const EngineParams& p, const TileInfo& ti, int i,
                                            int grow, const float (&v)[16], int cc,
                                            float* xchg) {
   const int m0 = cc * 16;
   if (p.epilogue == CQ_EPI_SWIGLU) {
-    if (i >= 64) {
+    // Tile rows i and i + 64 hold the gate and up value of output column
+    // rt * 64 + (i & 63).  The gate row finishes tokens 0-7 of the chunk and
+    // the up row tokens 8-15: each hands the other half over through xchg.
+    const int r = i & 63;
+    const bool up = i >= 64;
 #pragma unroll
-      for (int q = 0; q < 16; ++q) xchg[q * 64 + (i - 64)] = v[q];
+    for (int q = 0; q < 8; ++q) xchg[(up ? q : q + 8) * 64 + r] = up ? v[q] : v[q + 8];
+    named_bar_epilogue();
+    const int qb = up ? 8 : 0;
+    float h[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float other = xchg[(qb + q) * 64 + r];
+      const float mine = up ? v[q + 8] : v[q];
+      const float g = up ? other : mine;
+      const float u = up ? mine : other;
+      h[q] = g / (1.0f + __expf(-g)) * u;
     }
     named_bar_epilogue();
-    if (i < 64) {
-      const int col = ti.rt * 64 + i;
+    const int col = ti.rt * 64 + r;
+    const int mv = min(8, ti.m_valid - (m0 + qb));
+    if (col >= p.ldy) {
+      if (mv > 0) bad_access(23);
+    } else if (!p.out_rows) {
+      const int64_t r0 = static_cast<int64_t>(ti.x_row0) + m0 + qb;
+      if (mv > 0 && (r0 < 0 || r0 + mv > p.y_rows)) {
+        bad_access(23);
+      } else if (p.out_bf16) {
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.y) + r0 * p.ldy + col;
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const int m = m0 + q;
-        if (m < ti.m_valid) {
-          const float h = silu_f(v[q]) * xchg[q * 64 + i];
-          const int64_t orow = out_row(p, ti.x_row0 + m);
+        for (int q = 0; q < 8; ++q)
+          if (q < mv) dst[q * p.ldy] = __float2bfloat16_rn(h[q]);
+      } else {
+        float* dst = reinterpret_cast<float*>(p.y) + r0 * p.ldy + col;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < mv) dst[q * p.ldy] = h[q];
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q < mv) {
+          const int64_t orow = out_row(p, ti.x_row0 + m0 + qb + q);
           const int64_t off = orow * p.ldy + col;
-          if (orow < 0 || orow >= p.y_rows || col >= p.ldy) {
+          if (orow < 0 || orow >= p.y_rows) {
             bad_access(23);
           } else if (p.out_bf16)
-            reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(h);
+            reinterpret_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(h[q]);
           else
-            reinterpret_cast<float*>(p.y)[off] = h;
+            reinterpret_cast<float*>(p.y)[off] = h[q];
         }
       }
     }
-    named_bar_epilogue();
+  } else if (!p.out_rows) {
+    // tokens land in consecutive output rows: one bounds check per chunk and
+    // a strided store per token (the epilogue warps share their schedulers
+    // with the decoders, so few instructions per element matter)
+    if (grow < p.N) {
+      const int mv = min(16, ti.m_valid - m0);
+      const int64_t r0 = static_cast<int64_t>(ti.x_row0) + m0;
+      if (r0 < 0 || r0 + mv > p.y_rows || grow >= p.ldy) {
+        if (mv > 0) bad_access(23);
+      } else if (p.out_bf16) {
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.y) + r0 * p.ldy + grow;
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          if (q < mv) dst[q * p.ldy] = __float2bfloat16_rn(v[q]);
+      } else {
+        float* dst = reinterpret_cast<float*>(p.y) + r0 * p.ldy + grow;
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          if (q < mv) dst[q * p.ldy] = v[q];
+      }
+    }
   } else {
     if (grow < p.N) {
 #pragma unroll
@@ -626,9 +670,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int64_t x = r0; ok && x < r1;) {
         const Segment sg = segment_at(x, r1, p.spt);
-        const uint32_t db = seg & 1u;
+        const uint32_t db = C::NBUF == 2 ? (seg & 1u) : 0u;
+        const uint32_t duse = C::NBUF == 2 ? (seg >> 1) : seg;   // earlier uses of buffer db
         PROF_MARK();
-        if (!wait_phase(bar_dfree + 8 * db, ((seg >> 1) & 1u) ^ 1u, abort_flag, tmo,
+        if (!wait_phase(bar_dfree + 8 * db, (duse & 1u) ^ 1u, abort_flag, tmo,
                         SITE_MMA_DFREE)) {
           ok = false;
           break;
@@ -697,7 +742,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;                              // TMEM lane quarter
     const int half = warp >> 2;                          // which half of each slice
     const int i = q * 32 + lane;                         // tile row / TMEM lane
-    const uint32_t tid4 = 4u * i;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     uint32_t tgen = 0;                                   // table generations built
     int st = 0, ts = 0;
@@ -833,9 +877,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Segment sg = segment_at(x, r1, p.spt);
       const TileInfo ti = resolve_tile(p, sg.t, NT);
       const int grow = tile_row(p, ti.rt, i);
-      const uint32_t db = seg & 1u;
+      const uint32_t db = C::NBUF == 2 ? (seg & 1u) : 0u;
+      const uint32_t duse = C::NBUF == 2 ? (seg >> 1) : seg;
       PROF_MARK();
-      if (!wait_phase(bar_dfull + 8 * db, (seg >> 1) & 1u, abort_flag, tmo, SITE_DECODER_DFULL))
+      if (!wait_phase(bar_dfull + 8 * db, duse & 1u, abort_flag, tmo, SITE_DECODER_DFULL))
         ok = false;
       if (!vote_all_epilogue(ok)) {
         ok = false;

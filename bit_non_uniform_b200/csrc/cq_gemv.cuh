@@ -47,7 +47,6 @@
 
 #include "cq.h"
 #include "cq_device.cuh"
-#include "cq_engine.cuh"
 
 namespace cq {
 
@@ -268,7 +267,6 @@ __device__ __forceinline__ void gemv_cta(const GemvParams& p, const CUtensorMap*
   const int q_first = col0 >> 2;
   const int n_quads = ((col1 - 1) >> 2) - q_first + 1;
   const int n_loc = n_quads * p.spc;
-  const int T0 = q_first * p.spc;
 
   // ------------------------------------------------------------------ phase A
   if (tid == 0) {

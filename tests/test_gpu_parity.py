@@ -128,6 +128,10 @@ GEMM_CASES = [
     (129, 384,  1024, 2, 128, 0, 0, 0),
     (300, 256,  1536, 3, 512, 0, 1, 1),
     (17,  1152, 3072, 3, 512, 0, 1, 0),
+    # 256-token tiles (single-buffered accumulator): one exact tile, and three
+    # tiles with a ragged last one under the SwiGLU epilogue
+    (256, 384,  2048, 4, 256, 0, 0, 0),
+    (600, 256,  1024, 3, 128, 1, 1, 1),
 ]
 
 
@@ -305,6 +309,28 @@ def test_config3_w2_gate_up_swiglu(cq, M):
     check_swiglu(y, yr, bd, 0)
     y = cq.cq_gemm(x.cuda(), pk, sd, abd, N, K, B, G)
     check_gemm(y, yr, bd, f"config3 M={M} no epilogue")
+
+
+def test_swiglu_wide_tiles_sampled_columns(cq):
+    """The gate+up matrix with the SwiGLU epilogue at M = 4000: 256-token
+    tiles (single accumulator buffer, ragged last tile of 160 tokens), BF16
+    output; every token of a sample of output columns against the oracle's
+    gate and up rows."""
+    N, K, B, G, M = 6144, 7168, 2, 512, 4000
+    codes, s, ab = make_matrix(("config3",), N, K, B, G)
+    pk, sd, abd = to_dev(codes, s, ab, B, cq)
+    x = synthetic.activations(4321, M, K)
+    y = cq.cq_gemm(x.cuda(), pk, sd, abd, N, K, B, G, epilogue=cq.EPI_SWIGLU,
+                   out_dtype=cq.BF16).cpu()
+    torch.cuda.synchronize()
+    assert cq.device_error() == (0, 0)
+    n2 = N // 2
+    cols = np.sort(np.random.default_rng(7).choice(n2, 24, replace=False))
+    cols = np.unique(np.concatenate([cols, [0, 63, 64, n2 - 1]]))
+    rows = np.concatenate([cols, cols + n2])
+    po, so, ao = oracle_inputs(codes[rows], s[rows], ab[rows], B)
+    yr, bd = oracle.gemm(u16(x), po, so, ao, len(rows), K, B, G)
+    check_swiglu(y[:, cols], yr, bd, 1)
 
 
 @pytest.mark.parametrize("cfg,M", [("config2", 256), ("config3", 1024), ("config2", 4096)])
