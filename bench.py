@@ -61,7 +61,7 @@ WORKLOADS = {
 KERNEL_SOURCES = ("cq_gemv.cuh", "cq_gemv_launch.cuh", "cq_device.cuh")
 TRAFFIC = {
     "down_m1": {"kernel": "gemv_kernel<3,1>", "bytes": 8651776,
-                "sources_sha256": "a5eed5894780ada6febe7c8e501679bbda13e4754e7e44eb28999b674ff9c265"},
+                "sources_sha256": "9c0fd70674ae20b7b46b16200fe32c7edf8475c75be7cc9ec76340a56d490e7e"},
 }
 
 
