@@ -17,12 +17,14 @@
 //              banks) half each, then each turns its half of every 128-code
 //              slice into 32 BF16x2 words written to TMEM with tcgen05.st
 //              (the A operand of the MMA).
-//   warp 8     producer: 2-D TMA loads into a ring of shared-memory
-//              stages: per 128-code slice, two boxes of 64 weight rows x
-//              16*B bytes of packed codes (32-byte swizzle for W2, 64-byte
-//              for W4, none for W3's 48-byte rows, so the decoders'
-//              row-per-thread 16-byte reads are bank-conflict free), and the
-//              activation tile as 64-column boxes with the 128-byte swizzle.
+//   warp 8     producer, two lanes with two rings of shared-memory stages:
+//              lane 0 loads, per 128-code slice, two 2-D TMA boxes of 64
+//              weight rows x 16*B bytes of packed codes (32-byte swizzle for
+//              W2, 64-byte for W4, none for W3's 48-byte rows, so the
+//              decoders' row-per-thread 16-byte reads are bank-conflict
+//              free); lane 1 loads the activation tile as 64-column boxes
+//              with the 128-byte swizzle.  The code ring is deep and cheap,
+//              so the decoders run ahead of the activations.
 //   warp 9     TMEM owner and MMA issuer: tcgen05.mma kind::f16 with A from
 //              TMEM (decoded weights) and B from shared memory
 //              (activations), FP32 accumulators in TMEM, double-buffered so
@@ -64,17 +66,21 @@ struct EngineCfg {
   // tile's epilogue) while they fit beside the A ring, else one
   static constexpr int NBUF = kDCol + 2 * NT <= kTmemCols ? 2 : 1;
   static constexpr int SLICE_W_BYTES = kRows * 16 * 4;          // one slice of packed rows (B<=4)
-  static constexpr int W_BYTES = SPS * SLICE_W_BYTES;
-  static constexpr int X_BYTES = 256 * SPS * NT;                // 2*SPS boxes of 64 x NT bf16
-  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
+  static constexpr int W_STAGE = SPS * SLICE_W_BYTES;           // codes of SPS slices
+  static constexpr int X_STAGE = 256 * SPS * NT;                // 2*SPS boxes of 64 x NT bf16
   static constexpr int XCHG_BYTES = 16 * 64 * 4;
   static constexpr int MISC_BYTES = 1024;
   static constexpr int TBL_BYTES = 64 * 512;                    // static pair table (W3 size)
   static constexpr int BUDGET = 226 * 1024 - TBL_BYTES;         // dynamic part
-  static constexpr int S_RAW = (BUDGET - 1024 - XCHG_BYTES - MISC_BYTES) / STAGE_BYTES;
-  static constexpr int S = S_RAW > 6 ? 6 : S_RAW;
-  static constexpr int SMEM = 1024 + S * STAGE_BYTES + XCHG_BYTES + MISC_BYTES;
-  static_assert(S >= 2, "not enough shared memory for two stages");
+  static constexpr int AVAIL = BUDGET - 1024 - XCHG_BYTES - MISC_BYTES;
+  // two rings: activations (deep enough to cover the load latency) and codes
+  // (small stages, so the decoders can run ahead of the activations)
+  static constexpr int SX_RAW = (AVAIL - 2 * W_STAGE) / X_STAGE;
+  static constexpr int SX = SX_RAW > 4 ? 4 : SX_RAW;
+  static constexpr int SW_RAW = (AVAIL - SX * X_STAGE) / W_STAGE;
+  static constexpr int SW = SW_RAW > 8 ? 8 : SW_RAW;
+  static constexpr int SMEM = 1024 + SX * X_STAGE + SW * W_STAGE + XCHG_BYTES + MISC_BYTES;
+  static_assert(SX >= 2 && SW >= 2, "not enough shared memory for two stages per ring");
   static_assert(SMEM + TBL_BYTES <= 227 * 1024, "shared memory budget exceeded");
   static_assert(kDCol + NBUF * NT <= kTmemCols, "TMEM budget exceeded");
 };
@@ -512,16 +518,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   // 1024-align the working area (swizzled TMA destinations need it)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t stage0 = base;
-  const uint32_t xchg_s = stage0 + C::S * C::STAGE_BYTES;
+  const uint32_t xring = base;                             // [SX][X_STAGE]
+  const uint32_t wring = xring + C::SX * C::X_STAGE;       // [SW][W_STAGE]
+  const uint32_t xchg_s = wring + C::SW * C::W_STAGE;
   const uint32_t misc = xchg_s + C::XCHG_BYTES;
   uint8_t* const gbase = smem_raw + (base - raw);
   float* const xchg = reinterpret_cast<float*>(gbase + (xchg_s - base));
   uint32_t* const tbl = s_tbl;
   // barriers and flags
-  const uint32_t bar_full = misc;                         // [S]
-  const uint32_t bar_wempty = bar_full + 8 * C::S;        // [S]
-  const uint32_t bar_aready = bar_wempty + 8 * C::S;      // [4]
+  const uint32_t bar_wfull = misc;                        // [SW] codes landed
+  const uint32_t bar_wfree = bar_wfull + 8 * C::SW;       // [SW] decoders done with them
+  const uint32_t bar_xfull = bar_wfree + 8 * C::SW;       // [SX] activations landed
+  const uint32_t bar_xfree = bar_xfull + 8 * C::SX;       // [SX] MMAs done with them
+  const uint32_t bar_aready = bar_xfree + 8 * C::SX;      // [4]
   const uint32_t bar_tfree = bar_aready + 8 * kTmemRing;  // [4]
   const uint32_t bar_dfull = bar_tfree + 8 * kTmemRing;   // [2]
   const uint32_t bar_dfree = bar_dfull + 16;              // [2]
@@ -543,9 +552,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   long long prof_t = 0;
 
   if (tid == 0) {
-    for (int s = 0; s < C::S; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_wempty + 8 * s, kDecoders + 1);
+    for (int s = 0; s < C::SW; ++s) {
+      mbar_init(bar_wfull + 8 * s, 1);
+      mbar_init(bar_wfree + 8 * s, kDecoders);
+    }
+    for (int s = 0; s < C::SX; ++s) {
+      mbar_init(bar_xfull + 8 * s, 1);
+      mbar_init(bar_xfree + 8 * s, 1);
     }
     for (int s = 0; s < kTmemRing; ++s) {
       mbar_init(bar_aready + 8 * s, kDecoders);
@@ -590,77 +603,91 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
-    int st = 0;
-    uint32_t round = 0;
-    int load_no = 0;
-    for (int64_t x = r0; x < r1 && !*abort_flag;) {
-      const Segment sg = segment_at(x, r1, p.spt);
-      const TileInfo ti = resolve_tile(p, sg.t, NT);
-      const int Bw = ti.mat.B;
-      // first weight row of the two 64-row boxes of this tile
-      const int row_a = tile_row(p, ti.rt, 0);
-      const int row_b = tile_row(p, ti.rt, 64);
-      for (int sb = sg.s0; sb < sg.s1; sb += C::SPS) {
-        const int ns = (sg.s1 - sb) < C::SPS ? (sg.s1 - sb) : C::SPS;
-        PROF_MARK();
-        if (!wait_phase(bar_wempty + 8 * st, (round & 1u) ^ 1u, abort_flag, tmo,
-                        SITE_PRODUCER_EMPTY))
-          break;
-        PROF_ADD(0);
-        const bool skip = p.debug_skip_first_stage && load_no == 0;
-        // the kernel parameter's address is only ever used directly in the
-        // TMA instruction; table descriptors must lie inside the table
-        const bool map_ok =
-            !p.grouped || (ti.wmap >= &p.layer[0].map[0] && ti.wmap < &p.layer[p.E].map[0]);
-        if (!map_ok && lane == 0) bad_access(21);
-        if (!skip && map_ok && lane == 0) {
-          const uint32_t wbox = 64u * 16u * Bw;                   // bytes of one weight box
-          const uint32_t bytes = static_cast<uint32_t>(ns) * (2u * wbox) +
-                                 static_cast<uint32_t>(2 * ns * NT * 128);
-          const uint32_t wdst = stage0 + st * C::STAGE_BYTES;
-          const uint32_t xdst = wdst + C::W_BYTES;
-          mbar_arrive_expect_tx(bar_full + 8 * st, bytes);
-          for (int j = 0; j < ns; ++j) {
-            const int cb = (sb + j) * 16 * Bw;                   // byte column of the slice
-            const uint32_t sdst = wdst + j * C::SLICE_W_BYTES;
-            if (p.grouped) {
-              tma_load_2d(sdst, ti.wmap, cb, row_a, bar_full + 8 * st);
-              tma_load_2d(sdst + wbox, ti.wmap, cb, row_b, bar_full + 8 * st);
-            } else {
-              tma_load_2d(sdst, &wmap, cb, row_a, bar_full + 8 * st);
-              tma_load_2d(sdst + wbox, &wmap, cb, row_b, bar_full + 8 * st);
-            }
+    // Lane 0 keeps the code ring full, lane 1 the activation ring: the
+    // decoders run ahead of the activations (bounded by the TMEM ring) and
+    // the MMA waits for activations only.
+    if (lane < 2) {
+      const bool wl = lane == 0;
+      const int NS = wl ? C::SW : C::SX;
+      const uint32_t full0 = wl ? bar_wfull : bar_xfull;
+      const uint32_t free0 = wl ? bar_wfree : bar_xfree;
+      int st = 0;
+      uint32_t round = 0;
+      int load_no = 0;
+      for (int64_t x = r0; x < r1 && !*abort_flag;) {
+        const Segment sg = segment_at(x, r1, p.spt);
+        const TileInfo ti = resolve_tile(p, sg.t, NT);
+        const int Bw = ti.mat.B;
+        // first weight row of the two 64-row boxes of this tile
+        const int row_a = tile_row(p, ti.rt, 0);
+        const int row_b = tile_row(p, ti.rt, 64);
+        bool ok = true;
+        for (int sb = sg.s0; sb < sg.s1; sb += C::SPS) {
+          const int ns = (sg.s1 - sb) < C::SPS ? (sg.s1 - sb) : C::SPS;
+          PROF_MARK();
+          if (!wait_phase(free0 + 8 * st, (round & 1u) ^ 1u, abort_flag, tmo,
+                          SITE_PRODUCER_EMPTY)) {
+            ok = false;
+            break;
           }
-          for (int b = 0; b < 2 * ns; ++b)
-            tma_load_2d(xdst + b * (NT * 128), &xmap, sb * kSlice + b * 64, ti.x_row0,
-                        bar_full + 8 * st);
+          PROF_ADD(0);
+          const bool skip = p.debug_skip_first_stage && load_no == 0;
+          if (wl) {
+            // the kernel parameter's address is only ever used directly in the
+            // TMA instruction; table descriptors must lie inside the table
+            const bool map_ok = !p.grouped || (ti.wmap >= &p.layer[0].map[0] &&
+                                               ti.wmap < &p.layer[p.E].map[0]);
+            if (!map_ok) bad_access(21);
+            if (!skip && map_ok) {
+              const uint32_t wbox = 64u * 16u * Bw;                 // bytes of one weight box
+              const uint32_t wdst = wring + st * C::W_STAGE;
+              mbar_arrive_expect_tx(bar_wfull + 8 * st, static_cast<uint32_t>(ns) * 2u * wbox);
+              for (int j = 0; j < ns; ++j) {
+                const int cb = (sb + j) * 16 * Bw;                 // byte column of the slice
+                const uint32_t sdst = wdst + j * C::SLICE_W_BYTES;
+                if (p.grouped) {
+                  tma_load_2d(sdst, ti.wmap, cb, row_a, bar_wfull + 8 * st);
+                  tma_load_2d(sdst + wbox, ti.wmap, cb, row_b, bar_wfull + 8 * st);
+                } else {
+                  tma_load_2d(sdst, &wmap, cb, row_a, bar_wfull + 8 * st);
+                  tma_load_2d(sdst + wbox, &wmap, cb, row_b, bar_wfull + 8 * st);
+                }
+              }
+            }
+          } else if (!skip) {
+            const uint32_t xdst = xring + st * C::X_STAGE;
+            mbar_arrive_expect_tx(bar_xfull + 8 * st, static_cast<uint32_t>(2 * ns * NT * 128));
+            for (int b = 0; b < 2 * ns; ++b)
+              tma_load_2d(xdst + b * (NT * 128), &xmap, sb * kSlice + b * 64, ti.x_row0,
+                          bar_xfull + 8 * st);
+          }
+          PROF_ADD(1);
+          PROF_COUNT(2);
+          ++load_no;
+          if (++st == NS) {
+            st = 0;
+            ++round;
+          }
         }
-        __syncwarp();
-        PROF_ADD(1);
-        PROF_COUNT(2);
-        ++load_no;
-        if (++st == C::S) {
-          st = 0;
-          ++round;
+        if (!ok) break;
+        x = sg.end;
+      }
+      if (wl) PROF_FLUSH(8);
+      if (*abort_flag) {
+        // make sure no copy is still landing in shared memory before exit:
+        // the ring positions armed last are the only ones that may be in flight
+        const int armed = load_no < NS ? load_no : NS;
+        for (int k = 1; k <= armed; ++k) {
+          const int idx = load_no - k;
+          if (p.debug_skip_first_stage && idx == 0) continue;
+          const int sl = idx % NS;
+          const uint32_t rd = static_cast<uint32_t>(idx / NS);
+          volatile int dummy = 0;
+          mbar_wait(full0 + 8 * sl, rd & 1u, &dummy, tmo, SITE_TEARDOWN);
         }
       }
-      x = sg.end;
     }
-    if (lane == 0) PROF_FLUSH(8);
     __syncwarp();
-    if (lane == 0 && *abort_flag) {
-      // make sure no copy is still landing in shared memory before exit:
-      // the ring positions armed last are the only ones that may be in flight
-      const int armed = load_no < C::S ? load_no : C::S;
-      for (int k = 1; k <= armed; ++k) {
-        const int idx = load_no - k;
-        if (p.debug_skip_first_stage && idx == 0) continue;
-        const int s = idx % C::S;
-        const uint32_t rd = static_cast<uint32_t>(idx / C::S);
-        volatile int dummy = 0;
-        mbar_wait(bar_full + 8 * s, rd & 1u, &dummy, tmo, SITE_TEARDOWN);
-      }
-    }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -685,13 +712,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int sb = sg.s0; sb < sg.s1 && ok; sb += C::SPS) {
           const int ns = (sg.s1 - sb) < C::SPS ? (sg.s1 - sb) : C::SPS;
           PROF_MARK();
-          if (!wait_phase(bar_full + 8 * st, round & 1u, abort_flag, tmo, SITE_MMA_FULL)) {
+          if (!wait_phase(bar_xfull + 8 * st, round & 1u, abort_flag, tmo, SITE_MMA_FULL)) {
             ok = false;
             break;
           }
           PROF_ADD(1);
           tc_fence_after();
-          const uint64_t desc0 = smem_desc_sw128(stage0 + st * C::STAGE_BYTES + C::W_BYTES);
+          const uint64_t desc0 = smem_desc_sw128(xring + st * C::X_STAGE);
           for (int j = 0; j < ns; ++j) {
             PROF_MARK();
             if (!wait_phase(bar_aready + 8 * ts, tround & 1u, abort_flag, tmo,
@@ -719,8 +746,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (!ok) break;
-          mma_commit(bar_wempty + 8 * st);
-          if (++st == C::S) {
+          mma_commit(bar_xfree + 8 * st);
+          if (++st == C::SX) {
             st = 0;
             ++round;
           }
@@ -770,12 +797,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int sb = sg.s0; sb < sg.s1 && ok; sb += C::SPS) {
         const int ns = (sg.s1 - sb) < C::SPS ? (sg.s1 - sb) : C::SPS;
         PROF_MARK();
-        if (!wait_phase(bar_full + 8 * st, round & 1u, abort_flag, tmo, SITE_DECODER_FULL)) {
+        if (!wait_phase(bar_wfull + 8 * st, round & 1u, abort_flag, tmo, SITE_DECODER_FULL)) {
           ok = false;
           break;
         }
         PROF_ADD(0);
-        const uint32_t wrow = stage0 + st * C::STAGE_BYTES + i * 16 * Bw;
+        const uint32_t wrow = wring + st * C::W_STAGE + i * 16 * Bw;
         for (int j = 0; j < ns; ++j) {
           const int g = ((sb + j) * kSlice) / p.G;
           if (g != cur_g) {
@@ -856,8 +883,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        mbar_arrive(bar_wempty + 8 * st);
-        if (++st == C::S) {
+        mbar_arrive(bar_wfree + 8 * st);
+        if (++st == C::SW) {
           st = 0;
           ++round;
         }
