@@ -51,8 +51,7 @@ constexpr int kRows = 128;            // weight rows per tile (MMA M)
 constexpr int kSlice = 128;           // codes per slice along K
 constexpr int kThreads = 448;
 constexpr int kTmemCols = 512;
-constexpr int kTmemRing = 4;          // TMEM slice buffers (64 columns each)
-constexpr int kDCol = 256;            // first TMEM column of the accumulators
+constexpr int kTmemRing = 4;          // TMEM slice buffers (64 columns each), at most
 constexpr int kDecoders = 256;        // two threads per weight row
 constexpr int kEpilogue = 128;
 constexpr int kProducerWarp = 8;
@@ -62,9 +61,14 @@ constexpr int kEpiWarp0 = 10;
 template <int NT>
 struct EngineCfg {
   static constexpr int SPS = NT <= 32 ? 4 : (NT == 64 ? 2 : 1);   // slices per stage
-  // accumulator buffers in TMEM: two (the next tile's MMAs overlap this
-  // tile's epilogue) while they fit beside the A ring, else one
-  static constexpr int NBUF = kDCol + 2 * NT <= kTmemCols ? 2 : 1;
+  // TMEM: a ring of decoded slices (64 columns each) and the accumulators.
+  // Two accumulator buffers (the next tile's MMAs overlap this tile's
+  // epilogue) beside a ring of four slices while they fit, else beside a
+  // ring of two; at NT = 256 one buffer beside a ring of four.
+  static constexpr int FREE2 = (kTmemCols - 2 * NT) / 64;      // ring slots left by 2 buffers
+  static constexpr int NBUF = FREE2 >= 2 ? 2 : 1;
+  static constexpr int RING = FREE2 >= 4 ? 4 : (FREE2 >= 2 ? FREE2 : kTmemRing);
+  static constexpr int DCOL = RING * 64;                        // first accumulator column
   static constexpr int SLICE_W_BYTES = kRows * 16 * 4;          // one slice of packed rows (B<=4)
   static constexpr int W_STAGE = SPS * SLICE_W_BYTES;           // codes of SPS slices
   static constexpr int X_STAGE = 256 * SPS * NT;                // 2*SPS boxes of 64 x NT bf16
@@ -82,7 +86,7 @@ struct EngineCfg {
   static constexpr int SMEM = 1024 + SX * X_STAGE + SW * W_STAGE + XCHG_BYTES + MISC_BYTES;
   static_assert(SX >= 2 && SW >= 2, "not enough shared memory for two stages per ring");
   static_assert(SMEM + TBL_BYTES <= 227 * 1024, "shared memory budget exceeded");
-  static_assert(kDCol + NBUF * NT <= kTmemCols, "TMEM budget exceeded");
+  static_assert(DCOL + NBUF * NT <= kTmemCols && RING <= kTmemRing, "TMEM budget exceeded");
 };
 
 // One quantized matrix operand.
@@ -707,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         PROF_ADD(0);
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + kDCol + db * NT;
+        const uint32_t d_tmem = tmem_base + C::DCOL + db * NT;
         uint32_t acc = 0;
         for (int sb = sg.s0; sb < sg.s1 && ok; sb += C::SPS) {
           const int ns = (sg.s1 - sb) < C::SPS ? (sg.s1 - sb) : C::SPS;
@@ -740,7 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(bar_tfree + 8 * ts);
             PROF_ADD(3);
             PROF_COUNT(4);
-            if (++ts == kTmemRing) {
+            if (++ts == C::RING) {
               ts = 0;
               ++tround;
             }
@@ -877,7 +881,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bar_aready + 8 * ts);
           PROF_ADD(4);
           PROF_COUNT(6);
-          if (++ts == kTmemRing) {
+          if (++ts == C::RING) {
             ts = 0;
             ++tround;
           }
@@ -915,7 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       PROF_ADD(0);
       tc_fence_after();
-      const uint32_t daddr = tmem_base + lane_off + kDCol + db * NT;
+      const uint32_t daddr = tmem_base + lane_off + C::DCOL + db * NT;
       const int nchunks = (ti.m_valid + 15) >> 4;
       if (sg.s0 == 0 && sg.s1 == p.spt) {
         // whole tile in this CTA: straight to the output

@@ -11,17 +11,19 @@ namespace cq {
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;   // 2 s per wait
 
-// Token-tile width.  Each token tile decodes the weights again, and the
-// decode of a slice costs more than its MMAs up to N = 256, so wide problems
-// take the widest tile, as long as every CTA gets at least four 256-token
-// tiles: a 256-token tile has a single accumulator buffer in TMEM (the
-// epilogue stalls the MMAs), which only pays off over several tiles.
-static int pick_nt(int64_t M, int64_t n_rt, int sms) {
+// Token-tile width.  Each token tile decodes the weights again, and up to
+// N = 192 the decode of a slice costs more than its MMAs, so wide problems
+// take 192-token tiles (the widest with two accumulator buffers in TMEM,
+// beside a ring of two decoded slices) unless the ragged last tile wastes
+// more than 15% against 128-token tiles.  (256-token tiles leave room for a
+// single accumulator buffer: measured slower.)
+static int pick_nt(int64_t M) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
-  if (M <= 128 || ((M + 255) / 256) * n_rt < 4 * static_cast<int64_t>(sms)) return 128;
-  return 256;
+  if (M <= 128) return 128;
+  const int64_t pad192 = (M + 191) / 192 * 192, pad128 = (M + 127) / 128 * 128;
+  return pad192 * 100 <= pad128 * 115 ? 192 : 128;
 }
 
 struct GemmPlan {
@@ -33,7 +35,7 @@ static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int epilogue, int sms
   GemmPlan g;
   g.n_rt = epilogue == CQ_EPI_SWIGLU ? static_cast<int>(N / kRows)
                                      : static_cast<int>((N + kRows - 1) / kRows);
-  g.NT = pick_nt(M, g.n_rt, sms);
+  g.NT = pick_nt(M);
   g.n_tt = static_cast<int>((M + g.NT - 1) / g.NT);
   g.spt = static_cast<int>(K / kSlice);
   g.tiles = g.n_rt * g.n_tt;
@@ -142,7 +144,7 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
     case 32: return launch_engine<32>(p, map, wmap, stream);
     case 64: return launch_engine<64>(p, map, wmap, stream);
     case 128: return launch_engine<128>(p, map, wmap, stream);
-    default: return launch_engine<256>(p, map, wmap, stream);
+    default: return launch_engine<192>(p, map, wmap, stream);
   }
 }
 

@@ -128,8 +128,11 @@ GEMM_CASES = [
     (129, 384,  1024, 2, 128, 0, 0, 0),
     (300, 256,  1536, 3, 512, 0, 1, 1),
     (17,  1152, 3072, 3, 512, 0, 1, 0),
-    # 256-token tiles (single-buffered accumulator): one exact tile, and three
-    # tiles with a ragged last one under the SwiGLU epilogue
+    # 192-token tiles (two accumulator buffers beside a ring of two decoded
+    # slices): two tiles with a ragged second one, one ragged tile under the
+    # SwiGLU epilogue, and 128-token tiles where 192 would waste too much
+    (380, 384,  1024, 3, 256, 0, 0, 0),
+    (190, 256,  2048, 4, 512, 1, 1, 1),
     (256, 384,  2048, 4, 256, 0, 0, 0),
     (600, 256,  1024, 3, 128, 1, 1, 1),
 ]
@@ -312,10 +315,9 @@ def test_config3_w2_gate_up_swiglu(cq, M):
 
 
 def test_swiglu_wide_tiles_sampled_columns(cq):
-    """The gate+up matrix with the SwiGLU epilogue at M = 4000: 256-token
-    tiles (single accumulator buffer, ragged last tile of 160 tokens), BF16
-    output; every token of a sample of output columns against the oracle's
-    gate and up rows."""
+    """The gate+up matrix with the SwiGLU epilogue at M = 4000: 192-token
+    tiles (ragged last tile of 160 tokens), BF16 output; every token of a
+    sample of output columns against the oracle's gate and up rows."""
     N, K, B, G, M = 6144, 7168, 2, 512, 4000
     codes, s, ab = make_matrix(("config3",), N, K, B, G)
     pk, sd, abd = to_dev(codes, s, ab, B, cq)
