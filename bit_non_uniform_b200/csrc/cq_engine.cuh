@@ -52,13 +52,15 @@ constexpr int kSlice = 128;           // codes per slice along K
 constexpr int kThreads = 448;
 constexpr int kTmemCols = 512;
 constexpr int kTmemRing = 4;          // TMEM slice buffers (64 columns each), at most
-constexpr int kDecoders = 256;        // two threads per weight row
+constexpr int kDecoders = 256;        // two threads per weight row (even and odd slices)
 constexpr int kEpilogue = 128;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kEpiWarp0 = 10;
 
-template <int NT>
+// NT: token-tile width; TE: entries of a row's pair table (16 when every
+// matrix of the launch has B = 2 or 4, 64 when one may have B = 3).
+template <int NT, int TE>
 struct EngineCfg {
   static constexpr int SPS = NT <= 32 ? 4 : (NT == 64 ? 2 : 1);   // slices per stage
   // TMEM: a ring of decoded slices (64 columns each) and the accumulators.
@@ -74,18 +76,21 @@ struct EngineCfg {
   static constexpr int X_STAGE = 256 * SPS * NT;                // 2*SPS boxes of 64 x NT bf16
   static constexpr int XCHG_BYTES = 16 * 64 * 4;
   static constexpr int MISC_BYTES = 1024;
-  static constexpr int TBL_BYTES = 64 * 512;                    // static pair table (W3 size)
-  static constexpr int BUDGET = 226 * 1024 - TBL_BYTES;         // dynamic part
-  static constexpr int AVAIL = BUDGET - 1024 - XCHG_BYTES - MISC_BYTES;
+  static constexpr int TBL_BYTES = 2 * TE * kRows * 4;          // two pair tables per row
+  static constexpr int BUDGET = 226 * 1024;
+  static constexpr int AVAIL = BUDGET - 1024 - TBL_BYTES - XCHG_BYTES - MISC_BYTES;
   // two rings: activations (deep enough to cover the load latency) and codes
-  // (small stages, so the decoders can run ahead of the activations)
+  // (small stages, so the decoders can run ahead of the activations).  A
+  // finer activation ring (one box per entry) measured much slower: every
+  // TMA operation has a fixed issue cost.
   static constexpr int SX_RAW = (AVAIL - 2 * W_STAGE) / X_STAGE;
   static constexpr int SX = SX_RAW > 4 ? 4 : SX_RAW;
   static constexpr int SW_RAW = (AVAIL - SX * X_STAGE) / W_STAGE;
   static constexpr int SW = SW_RAW > 8 ? 8 : SW_RAW;
-  static constexpr int SMEM = 1024 + SX * X_STAGE + SW * W_STAGE + XCHG_BYTES + MISC_BYTES;
+  static constexpr int SMEM =
+      1024 + SX * X_STAGE + SW * W_STAGE + TBL_BYTES + XCHG_BYTES + MISC_BYTES;
   static_assert(SX >= 2 && SW >= 2, "not enough shared memory for two stages per ring");
-  static_assert(SMEM + TBL_BYTES <= 227 * 1024, "shared memory budget exceeded");
+  static_assert(SMEM <= 227 * 1024, "shared memory budget exceeded");
   static_assert(DCOL + NBUF * NT <= kTmemCols && RING <= kTmemRing, "TMEM budget exceeded");
 };
 
@@ -326,6 +331,14 @@ __device__ __forceinline__ void build_table(uint32_t* tbl, int i, bool valid, fl
   }
 }
 
+// Build the whole pair table of tile row i (every entry), levels as above.
+template <int B>
+__device__ __forceinline__ void build_table_all(uint32_t* tbl, int i, bool valid, float s,
+                                                uint32_t abw, int mode) {
+  build_table<B, 0>(tbl, i, valid, s, abw, mode);
+  build_table<B, 1>(tbl, i, valid, s, abw, mode);
+}
+
 // Bits [sh, ...) of word w moved to bit 7 (the table's entry stride in words).
 __device__ __forceinline__ uint32_t at_bit7(uint32_t w, int sh) {
   return sh >= 7 ? (w >> (sh - 7)) : (w << (7 - sh));
@@ -511,24 +524,24 @@ __device__ __forceinline__ void finalize16(const EngineParams& p, const TileInfo
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <int NT>
+template <int NT, int TE>
 __global__ void __launch_bounds__(kThreads, 1)
     engine_kernel(const __grid_constant__ EngineParams p,
                   const __grid_constant__ CUtensorMap xmap,
                   const __grid_constant__ CUtensorMap wmap) {
-  using C = EngineCfg<NT>;
-  __shared__ __align__(32768) uint32_t s_tbl[64 * kRows];   // per-row pair tables
+  using C = EngineCfg<NT, TE>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-align the working area (swizzled TMA destinations need it)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   const uint32_t xring = base;                             // [SX][X_STAGE]
   const uint32_t wring = xring + C::SX * C::X_STAGE;       // [SW][W_STAGE]
-  const uint32_t xchg_s = wring + C::SW * C::W_STAGE;
+  const uint32_t tbl_s = wring + C::SW * C::W_STAGE;       // [2][TE][128] words
+  const uint32_t xchg_s = tbl_s + C::TBL_BYTES;
   const uint32_t misc = xchg_s + C::XCHG_BYTES;
   uint8_t* const gbase = smem_raw + (base - raw);
   float* const xchg = reinterpret_cast<float*>(gbase + (xchg_s - base));
-  uint32_t* const tbl = s_tbl;
+  uint32_t* const tbl = reinterpret_cast<uint32_t*>(gbase + (tbl_s - base));
   // barriers and flags
   const uint32_t bar_wfull = misc;                        // [SW] codes landed
   const uint32_t bar_wfree = bar_wfull + 8 * C::SW;       // [SW] decoders done with them
@@ -539,9 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_dfull = bar_tfree + 8 * kTmemRing;   // [2]
   const uint32_t bar_dfree = bar_dfull + 16;              // [2]
   const uint32_t bar_fin = bar_dfree + 16;
-  const uint32_t bar_tdone = bar_fin + 8;                 // [4] per lane quarter
-  const uint32_t bar_tready = bar_tdone + 32;             // [4]
-  const uint32_t slot_tmem = bar_tready + 32;
+  const uint32_t slot_tmem = bar_fin + 8;
   volatile int* const abort_flag =
       reinterpret_cast<volatile int*>(gbase + (slot_tmem + 8 - base));
   volatile int* const last_flag =
@@ -565,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_xfree + 8 * s, 1);
     }
     for (int s = 0; s < kTmemRing; ++s) {
-      mbar_init(bar_aready + 8 * s, kDecoders);
+      mbar_init(bar_aready + 8 * s, kRows);          // one decoder thread per row and slice
       mbar_init(bar_tfree + 8 * s, 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -573,10 +584,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_dfree + 8 * s, kEpilogue);
     }
     mbar_init(bar_fin, 1);
-    for (int s = 0; s < 4; ++s) {
-      mbar_init(bar_tdone + 8 * s, 64);
-      mbar_init(bar_tready + 8 * s, 64);
-    }
     *abort_flag = 0;
     *last_flag = 0;
     fence_mbar_init();
@@ -607,9 +614,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
-    // Lane 0 keeps the code ring full, lane 1 the activation ring: the
-    // decoders run ahead of the activations (bounded by the TMEM ring) and
-    // the MMA waits for activations only.
+    // Lane 0 keeps the code ring full, lane 1 the activation ring (both in
+    // stages of SPS slices): the decoders run ahead of the activations
+    // (bounded by the TMEM ring) and the MMA waits for activations only.
     if (lane < 2) {
       const bool wl = lane == 0;
       const int NS = wl ? C::SW : C::SX;
@@ -618,63 +625,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       int st = 0;
       uint32_t round = 0;
       int load_no = 0;
-      for (int64_t x = r0; x < r1 && !*abort_flag;) {
+      bool ok = true;
+      for (int64_t x = r0; ok && x < r1 && !*abort_flag;) {
         const Segment sg = segment_at(x, r1, p.spt);
         const TileInfo ti = resolve_tile(p, sg.t, NT);
         const int Bw = ti.mat.B;
         // first weight row of the two 64-row boxes of this tile
         const int row_a = tile_row(p, ti.rt, 0);
         const int row_b = tile_row(p, ti.rt, 64);
-        bool ok = true;
-        for (int sb = sg.s0; sb < sg.s1; sb += C::SPS) {
+        for (int sb = sg.s0; ok && sb < sg.s1; sb += C::SPS) {
           const int ns = (sg.s1 - sb) < C::SPS ? (sg.s1 - sb) : C::SPS;
-          PROF_MARK();
-          if (!wait_phase(free0 + 8 * st, (round & 1u) ^ 1u, abort_flag, tmo,
-                          SITE_PRODUCER_EMPTY)) {
-            ok = false;
-            break;
-          }
-          PROF_ADD(0);
-          const bool skip = p.debug_skip_first_stage && load_no == 0;
-          if (wl) {
-            // the kernel parameter's address is only ever used directly in the
-            // TMA instruction; table descriptors must lie inside the table
-            const bool map_ok = !p.grouped || (ti.wmap >= &p.layer[0].map[0] &&
-                                               ti.wmap < &p.layer[p.E].map[0]);
-            if (!map_ok) bad_access(21);
-            if (!skip && map_ok) {
-              const uint32_t wbox = 64u * 16u * Bw;                 // bytes of one weight box
-              const uint32_t wdst = wring + st * C::W_STAGE;
-              mbar_arrive_expect_tx(bar_wfull + 8 * st, static_cast<uint32_t>(ns) * 2u * wbox);
-              for (int j = 0; j < ns; ++j) {
-                const int cb = (sb + j) * 16 * Bw;                 // byte column of the slice
-                const uint32_t sdst = wdst + j * C::SLICE_W_BYTES;
-                if (p.grouped) {
-                  tma_load_2d(sdst, ti.wmap, cb, row_a, bar_wfull + 8 * st);
-                  tma_load_2d(sdst + wbox, ti.wmap, cb, row_b, bar_wfull + 8 * st);
-                } else {
-                  tma_load_2d(sdst, &wmap, cb, row_a, bar_wfull + 8 * st);
-                  tma_load_2d(sdst + wbox, &wmap, cb, row_b, bar_wfull + 8 * st);
+          {
+            PROF_MARK();
+            if (!wait_phase(free0 + 8 * st, (round & 1u) ^ 1u, abort_flag, tmo,
+                            SITE_PRODUCER_EMPTY)) {
+              ok = false;
+              break;
+            }
+            PROF_ADD(0);
+            const bool skip = p.debug_skip_first_stage && load_no == 0;
+            if (wl) {
+              // the kernel parameter's address is only ever used directly in
+              // the TMA instruction; table descriptors must lie inside the table
+              const bool map_ok = !p.grouped || (ti.wmap >= &p.layer[0].map[0] &&
+                                                 ti.wmap < &p.layer[p.E].map[0]);
+              if (!map_ok) bad_access(21);
+              if (!skip && map_ok) {
+                const uint32_t wbox = 64u * 16u * Bw;               // bytes of one weight box
+                const uint32_t wdst = wring + st * C::W_STAGE;
+                mbar_arrive_expect_tx(bar_wfull + 8 * st, static_cast<uint32_t>(ns) * 2u * wbox);
+                for (int j = 0; j < ns; ++j) {
+                  const int cb = (sb + j) * 16 * Bw;               // byte column of the slice
+                  const uint32_t sdst = wdst + j * C::SLICE_W_BYTES;
+                  if (p.grouped) {
+                    tma_load_2d(sdst, ti.wmap, cb, row_a, bar_wfull + 8 * st);
+                    tma_load_2d(sdst + wbox, ti.wmap, cb, row_b, bar_wfull + 8 * st);
+                  } else {
+                    tma_load_2d(sdst, &wmap, cb, row_a, bar_wfull + 8 * st);
+                    tma_load_2d(sdst + wbox, &wmap, cb, row_b, bar_wfull + 8 * st);
+                  }
                 }
               }
+            } else if (!skip) {
+              const uint32_t xdst = xring + st * C::X_STAGE;
+              mbar_arrive_expect_tx(bar_xfull + 8 * st, static_cast<uint32_t>(2 * ns * NT * 128));
+              for (int b = 0; b < 2 * ns; ++b)
+                tma_load_2d(xdst + b * (NT * 128), &xmap, sb * kSlice + b * 64, ti.x_row0,
+                            bar_xfull + 8 * st);
             }
-          } else if (!skip) {
-            const uint32_t xdst = xring + st * C::X_STAGE;
-            mbar_arrive_expect_tx(bar_xfull + 8 * st, static_cast<uint32_t>(2 * ns * NT * 128));
-            for (int b = 0; b < 2 * ns; ++b)
-              tma_load_2d(xdst + b * (NT * 128), &xmap, sb * kSlice + b * 64, ti.x_row0,
-                          bar_xfull + 8 * st);
-          }
-          PROF_ADD(1);
-          PROF_COUNT(2);
-          ++load_no;
-          if (++st == NS) {
-            st = 0;
-            ++round;
+            PROF_ADD(1);
+            PROF_COUNT(2);
+            ++load_no;
+            if (++st == NS) {
+              st = 0;
+              ++round;
+            }
           }
         }
-        if (!ok) break;
-        x = sg.end;
+        if (ok) x = sg.end;
       }
       if (wl) PROF_FLUSH(8);
       if (*abort_flag) {
@@ -770,15 +778,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ decoders
+    // Warp q (q < 4) decodes the even slices and warp q + 4 the odd ones,
+    // each slice whole, for tile rows 32q .. 32q+31 (TMEM lanes).  Each of
+    // the two has its own pair table per row, so neither waits for the other.
     const int q = warp & 3;                              // TMEM lane quarter
-    const int half = warp >> 2;                          // which half of each slice
+    const int h = warp >> 2;                             // parity of the slices decoded
     const int i = q * 32 + lane;                         // tile row / TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    uint32_t tgen = 0;                                   // table generations built
+    uint32_t* const mytbl = tbl + h * (TE * kRows);
     int st = 0, ts = 0;
     uint32_t round = 0, tround = 0;
     bool ok = true;
     const int ng = p.K / p.G;
+    const int spc = p.G / kSlice;                        // slices per group
     for (int64_t x = r0; ok && x < r1;) {
       const Segment sg = segment_at(x, r1, p.spt);
       const TileInfo ti = resolve_tile(p, sg.t, NT);
@@ -787,16 +799,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // 16-byte chunk v of this row sits at chunk (v ^ swz) of the row (TMA swizzle)
       const uint32_t swz = Bw == 2 ? ((i >> 2) & 1u) : (Bw == 4 ? ((i >> 1) & 3u) : 0u);
       const bool valid = grow < p.N;
-      // group metadata: the current group and a prefetch of the next one
+      // group metadata: the current group and a prefetch of the next group
+      // this thread meets (its first slice of this segment, then after each
+      // switch the group of its first slice past the current group)
       int cur_g = -1;
-      int g_next = (sg.s0 * kSlice) / p.G;
+      const int s_first = sg.s0 + ((sg.s0 & 1) != h ? 1 : 0);
       float s_next = 0.f;
       uint32_t ab_next = 0;
-      if (valid && g_next < ng) {
-        s_next = __ldg(ti.mat.scales + static_cast<int64_t>(grow) * ng + g_next);
-        ab_next = __ldg(ti.mat.ab + static_cast<int64_t>(grow) * ng + g_next);
-      } else if (valid) {
-        bad_access(22);
+      if (valid && s_first < sg.s1) {
+        const int g0 = s_first / spc;
+        if (g0 < ng) {
+          s_next = __ldg(ti.mat.scales + static_cast<int64_t>(grow) * ng + g0);
+          ab_next = __ldg(ti.mat.ab + static_cast<int64_t>(grow) * ng + g0);
+        } else {
+          bad_access(22);
+        }
       }
       for (int sb = sg.s0; sb < sg.s1 && ok; sb += C::SPS) {
         const int ns = (sg.s1 - sb) < C::SPS ? (sg.s1 - sb) : C::SPS;
@@ -808,79 +825,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         PROF_ADD(0);
         const uint32_t wrow = wring + st * C::W_STAGE + i * 16 * Bw;
         for (int j = 0; j < ns; ++j) {
-          const int g = ((sb + j) * kSlice) / p.G;
-          if (g != cur_g) {
-            // g == g_next here: slices visit groups in order
-            const float s_cur = s_next;
-            const uint32_t ab_cur = ab_next;
-            cur_g = g;
-            g_next = g + 1;
-            if (valid && g_next < ng) {
-              s_next = __ldg(ti.mat.scales + static_cast<int64_t>(grow) * ng + g_next);
-              ab_next = __ldg(ti.mat.ab + static_cast<int64_t>(grow) * ng + g_next);
+          const int sl = sb + j;
+          if ((sl & 1) == h) {
+            const int g = sl / spc;
+            if (TE < 64 && Bw == 3) {
+              // a 64-entry table does not fit this launch's tables (the host
+              // never plans it): record it and leave the table alone
+              if (g != cur_g && i == 0) bad_access(27);
+              cur_g = g;
             }
-            // both threads of the row are done with the old table ...
-            mbar_arrive(bar_tdone + 8 * q);
-            if (!wait_phase(bar_tdone + 8 * q, tgen & 1u, abort_flag, tmo, SITE_TABLE)) {
+            if (g != cur_g) {
+              // slices of this parity visit groups in order: g is the
+              // prefetched one
+              const float s_cur = s_next;
+              const uint32_t ab_cur = ab_next;
+              cur_g = g;
+              const int send = (g + 1) * spc;                 // first slice past group g
+              const int snext = send + ((send & 1) != h ? 1 : 0);
+              const int gn = snext / spc;
+              if (valid && snext < sg.s1 && gn < ng) {
+                s_next = __ldg(ti.mat.scales + static_cast<int64_t>(grow) * ng + gn);
+                ab_next = __ldg(ti.mat.ab + static_cast<int64_t>(grow) * ng + gn);
+              }
+              if (Bw == 2)
+                build_table_all<2>(mytbl, i, valid, s_cur, ab_cur, p.mode);
+              else if (Bw == 3)
+                build_table_all<3>(mytbl, i, valid, s_cur, ab_cur, p.mode);
+              else
+                build_table_all<4>(mytbl, i, valid, s_cur, ab_cur, p.mode);
+              PROF_COUNT(7);
+            }
+            PROF_ADD(1);
+            if (!wait_phase(bar_tfree + 8 * ts, (tround & 1u) ^ 1u, abort_flag, tmo,
+                            SITE_DECODER_TFREE)) {
               ok = false;
               break;
             }
-            if (half == 0) {
-              if (Bw == 2)
-                build_table<2, 0>(tbl, i, valid, s_cur, ab_cur, p.mode);
-              else if (Bw == 3)
-                build_table<3, 0>(tbl, i, valid, s_cur, ab_cur, p.mode);
-              else
-                build_table<4, 0>(tbl, i, valid, s_cur, ab_cur, p.mode);
+            PROF_ADD(2);
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + lane_off + ts * 64;
+            const uint4* caddr =
+                reinterpret_cast<const uint4*>(gbase + (wrow + j * C::SLICE_W_BYTES - base));
+            if (Bw == 2) {
+              decode_half_slice_to_tmem<2, 0>(caddr, swz, mytbl, i, taddr);
+              decode_half_slice_to_tmem<2, 1>(caddr, swz, mytbl, i, taddr + 32);
+            } else if (Bw == 3) {
+              decode_half_slice_to_tmem<3, 0>(caddr, swz, mytbl, i, taddr);
+              decode_half_slice_to_tmem<3, 1>(caddr, swz, mytbl, i, taddr + 32);
             } else {
-              if (Bw == 2)
-                build_table<2, 1>(tbl, i, valid, s_cur, ab_cur, p.mode);
-              else if (Bw == 3)
-                build_table<3, 1>(tbl, i, valid, s_cur, ab_cur, p.mode);
-              else
-                build_table<4, 1>(tbl, i, valid, s_cur, ab_cur, p.mode);
+              decode_half_slice_to_tmem<4, 0>(caddr, swz, mytbl, i, taddr);
+              decode_half_slice_to_tmem<4, 1>(caddr, swz, mytbl, i, taddr + 32);
             }
-            // ... and both halves of the new one are written
-            mbar_arrive(bar_tready + 8 * q);
-            if (!wait_phase(bar_tready + 8 * q, tgen & 1u, abort_flag, tmo, SITE_TABLE)) {
-              ok = false;
-              break;
-            }
-            ++tgen;
-            PROF_COUNT(7);
+            PROF_ADD(3);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar_aready + 8 * ts);
+            PROF_ADD(4);
+            PROF_COUNT(6);
           }
-          PROF_ADD(1);
-          if (!wait_phase(bar_tfree + 8 * ts, (tround & 1u) ^ 1u, abort_flag, tmo,
-                          SITE_DECODER_TFREE)) {
-            ok = false;
-            break;
-          }
-          PROF_ADD(2);
-          tc_fence_after();
-          const uint32_t taddr = tmem_base + lane_off + ts * 64 + 32 * half;
-          const uint4* caddr =
-              reinterpret_cast<const uint4*>(gbase + (wrow + j * C::SLICE_W_BYTES - base));
-          if (half == 0) {
-            if (Bw == 2)
-              decode_half_slice_to_tmem<2, 0>(caddr, swz, tbl, i, taddr);
-            else if (Bw == 3)
-              decode_half_slice_to_tmem<3, 0>(caddr, swz, tbl, i, taddr);
-            else
-              decode_half_slice_to_tmem<4, 0>(caddr, swz, tbl, i, taddr);
-          } else {
-            if (Bw == 2)
-              decode_half_slice_to_tmem<2, 1>(caddr, swz, tbl, i, taddr);
-            else if (Bw == 3)
-              decode_half_slice_to_tmem<3, 1>(caddr, swz, tbl, i, taddr);
-            else
-              decode_half_slice_to_tmem<4, 1>(caddr, swz, tbl, i, taddr);
-          }
-          PROF_ADD(3);
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(bar_aready + 8 * ts);
-          PROF_ADD(4);
-          PROF_COUNT(6);
           if (++ts == C::RING) {
             ts = 0;
             ++tround;

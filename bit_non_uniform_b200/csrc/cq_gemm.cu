@@ -14,16 +14,17 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;   // 2 s per wait
 // Token-tile width.  Each token tile decodes the weights again, and up to
 // N = 192 the decode of a slice costs more than its MMAs, so wide problems
 // take 192-token tiles (the widest with two accumulator buffers in TMEM,
-// beside a ring of two decoded slices) unless the ragged last tile wastes
-// more than 15% against 128-token tiles.  (256-token tiles leave room for a
-// single accumulator buffer: measured slower.)
-static int pick_nt(int64_t M) {
+// beside a ring of two decoded slices) unless the ragged last tile pads too
+// much against 128-token tiles: 15%, or 5% for W3, whose 64-entry pair
+// tables leave room for only two 192-token activation stages.  (256-token
+// tiles leave room for a single accumulator buffer: measured slower.)
+static int pick_nt(int64_t M, int B) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
   if (M <= 128) return 128;
   const int64_t pad192 = (M + 191) / 192 * 192, pad128 = (M + 127) / 128 * 128;
-  return pad192 * 100 <= pad128 * 115 ? 192 : 128;
+  return pad192 * 100 <= pad128 * (B == 3 ? 105 : 115) ? 192 : 128;
 }
 
 struct GemmPlan {
@@ -31,11 +32,11 @@ struct GemmPlan {
   size_t ws_counter_bytes, ws_partial_bytes;
 };
 
-static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int epilogue, int sms) {
+static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int B, int epilogue, int sms) {
   GemmPlan g;
   g.n_rt = epilogue == CQ_EPI_SWIGLU ? static_cast<int>(N / kRows)
                                      : static_cast<int>((N + kRows - 1) / kRows);
-  g.NT = pick_nt(M);
+  g.NT = pick_nt(M, B);
   g.n_tt = static_cast<int>((M + g.NT - 1) / g.NT);
   g.spt = static_cast<int>(K / kSlice);
   g.tiles = g.n_rt * g.n_tt;
@@ -55,7 +56,7 @@ static void gemm_scratch(int64_t M, int64_t N, int64_t K, int B, int G, int epil
     *total = v.ws_counter_bytes + v.ws_partial_bytes;
     return;
   }
-  const GemmPlan g = plan_gemm(M, N, K, epilogue, sms);
+  const GemmPlan g = plan_gemm(M, N, K, B, epilogue, sms);
   *counter_bytes = g.ws_counter_bytes;
   *total = g.ws_counter_bytes + g.ws_partial_bytes;
 }
@@ -63,19 +64,28 @@ static void gemm_scratch(int64_t M, int64_t N, int64_t K, int B, int G, int epil
 // ---------------------------------------------------------------------------
 // tensor-core engine path
 // ---------------------------------------------------------------------------
-template <int NT>
+template <int NT, int TE>
 static int launch_engine(const EngineParams& p, const CUtensorMap& map, const CUtensorMap& wmap,
                          cudaStream_t s) {
-  using C = EngineCfg<NT>;
+  using C = EngineCfg<NT, TE>;
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(engine_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(engine_kernel<NT, TE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM) != cudaSuccess)
       return CQ_ERR_CUDA;
     attr_set = true;
   }
-  engine_kernel<NT><<<p.P, kThreads, C::SMEM, s>>>(p, map, wmap);
+  engine_kernel<NT, TE><<<p.P, kThreads, C::SMEM, s>>>(p, map, wmap);
   return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+// Pair tables of 64 entries for W3, 16 for W2/W4 (the smaller tables leave
+// room for more activation stages).
+template <int NT>
+static int launch_engine_te(const EngineParams& p, const CUtensorMap& map,
+                            const CUtensorMap& wmap, int B, cudaStream_t s) {
+  if (B == 3) return launch_engine<NT, 64>(p, map, wmap, s);
+  return launch_engine<NT, 16>(p, map, wmap, s);
 }
 
 int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* scales,
@@ -100,7 +110,7 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
   if (v.use)
     return run_gemv(v, x, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype, y,
                     stream, timeout_ns, trace);
-  const GemmPlan g = plan_gemm(M, N, K, epilogue, sms);
+  const GemmPlan g = plan_gemm(M, N, K, B, epilogue, sms);
   const size_t need = g.ws_counter_bytes + g.ws_partial_bytes;
   if (ws_bytes < need || (need && !workspace)) return CQ_ERR_WORKSPACE;
   if (!aligned(workspace, 16)) return CQ_ERR_UNSUPPORTED;
@@ -140,11 +150,11 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
   p.trace = trace;
 
   switch (g.NT) {
-    case 16: return launch_engine<16>(p, map, wmap, stream);
-    case 32: return launch_engine<32>(p, map, wmap, stream);
-    case 64: return launch_engine<64>(p, map, wmap, stream);
-    case 128: return launch_engine<128>(p, map, wmap, stream);
-    default: return launch_engine<192>(p, map, wmap, stream);
+    case 16: return launch_engine_te<16>(p, map, wmap, B, stream);
+    case 32: return launch_engine_te<32>(p, map, wmap, B, stream);
+    case 64: return launch_engine_te<64>(p, map, wmap, B, stream);
+    case 128: return launch_engine_te<128>(p, map, wmap, B, stream);
+    default: return launch_engine_te<192>(p, map, wmap, B, stream);
   }
 }
 

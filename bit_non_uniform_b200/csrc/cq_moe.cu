@@ -322,7 +322,7 @@ template <int NT>
 static int launch_grouped(const EngineParams& p, const CUtensorMap& xmap, cudaStream_t s) {
   CUtensorMap unused;
   memset(&unused, 0, sizeof(unused));
-  return launch_engine<NT>(p, xmap, unused, s);
+  return launch_engine<NT, 64>(p, xmap, unused, s);   // experts may mix bit widths
 }
 
 static int launch_grouped_nt(int NT, const EngineParams& p, const CUtensorMap& xmap,
