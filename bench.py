@@ -81,13 +81,30 @@ def measured_traffic(name):
     return rec["bytes"]
 
 
+def main_roofline(r, ach_gbs, hbm, tf_burst, traffic, name, peak_src):
+    """The roofline of the main line's kernel: HBM for the decode-sized
+    workloads, the BF16 tensor peak (burst: one kernel timed alone) for
+    M >= 256."""
+    if r["M"] >= 256:
+        return {"bound": "tensor", "achieved": round(r["tflops"], 1), "peak": tf_burst,
+                "unit": "TFLOP/s", "frac": round(r["tflops"] / tf_burst, 4), "traffic": traffic,
+                "kernel": dominant_kernel(name), "peak_source": peak_src}
+    return {"bound": "hbm", "achieved": round(ach_gbs, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(ach_gbs / hbm, 4), "traffic": traffic,
+            "kernel": dominant_kernel(name), "peak_source": peak_src}
+
+
 def dominant_kernel(name):
     """The kernel one cq_gemm launch of the workload runs (the only one it runs)."""
     _, N, K, B, G, M, epi = WORKLOADS[name]
     if M <= 2:
         return f"gemv_kernel<{B},{M}>"
-    nt = 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
-    return f"engine_kernel<{nt}>"
+    if M <= 128:
+        nt = 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
+    else:
+        pad192, pad128 = -(-M // 192) * 192, -(-M // 128) * 128
+        nt = 192 if pad192 * 100 <= pad128 * (105 if B == 3 else 115) else 128
+    return f"engine_kernel<{nt},{64 if B == 3 else 16}>"
 
 
 def packed_bytes(N, K, B, G):
@@ -579,9 +596,7 @@ def main():
                    "l2": f"inputs larger than L2: {r['R']} rotating weight copies, "
                          f"{r['rot_mb']:.0f} MB",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(ach / hbm, 4), "traffic": traffic,
-                     "kernel": dominant_kernel(args.workload), "peak_source": peak_src},
+        "roofline": main_roofline(r, ach, hbm, tf_burst, traffic, args.workload, peak_src),
         "e2e": e2e,
         "gpu_launches": args.steps,
         "clocks": r["clocks"],
