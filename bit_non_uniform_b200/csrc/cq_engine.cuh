@@ -187,7 +187,7 @@ struct TileInfo {
   int m_valid;      // valid tokens in this tile (<= NT)
 };
 
-// Tile t of the launch.  Plain mode: t = rt * n_tt + tt.  Grouped mode:
+// Tile t of the launch.  Plain mode: t = tt * n_rt + rt.  Grouped mode:
 // experts in order, each contributing n_rt x ntt(e) tiles (tt fastest), so
 // expert e owns tiles [n_rt * ttpre[e], n_rt * ttpre[e+1]).
 __device__ __forceinline__ TileInfo resolve_tile(const EngineParams& p, int t, int NT) {
@@ -195,8 +195,10 @@ __device__ __forceinline__ TileInfo resolve_tile(const EngineParams& p, int t, i
   if (!p.grouped) {
     ti.mat = p.mat;
     ti.wmap = nullptr;          // plain mode loads through the kernel's own parameter
-    ti.rt = t / p.n_tt;
-    ti.tt = t - ti.rt * p.n_tt;
+    // token tiles outermost: CTAs working at the same time share activation
+    // tiles, which then stay in L2 (all row tiles' weights fit there anyway)
+    ti.tt = t / p.n_rt;
+    ti.rt = t - ti.tt * p.n_rt;
     ti.x_row0 = ti.tt * NT;
     const int rem = p.M - ti.x_row0;
     ti.m_valid = rem < NT ? rem : NT;
