@@ -168,3 +168,37 @@ def test_config5_prefill_layer_sampled(cq):
     comb = (w[tk].double().cuda()[:, :, None] * ro.view(T, k, H)[tk].double()).sum(1)
     assert torch.allclose(out[tk].double(), comb, rtol=1e-6, atol=1e-6)
     del experts, layer
+
+
+def test_moe_degenerate_layers(cq):
+    """Degenerate routing: one expert with k = 1 (every token on it, the
+    decode-sized path), every route dropped (all outputs zero), and an empty
+    batch (nothing launched)."""
+    H, I, G, B = 512, 256, 128, 3
+    tag = ("degenerate",)
+    experts = [expert_gpu(cq, tag, 0, B, H, I, G)]
+    layer = cq.moe_prepare_layer(experts, H, I, G)
+    # one expert, top-1, three tokens
+    T = 3
+    x = synthetic.activations(77, T, H)
+    ids = torch.zeros((T, 1), dtype=torch.int32)
+    w = torch.ones((T, 1), dtype=torch.float32)
+    ro, out = cq.cq_moe_grouped_gemm(x.cuda(), ids.cuda(), w.cuda(), layer, 1, H, I, G)
+    torch.cuda.synchronize()
+    assert cq.device_error() == (0, 0)
+    oexp = {0: expert_oracle(tag, 0, B, H, I, G)}
+    ref = oracle.moe_routes(u16(x), ids.numpy(), oexp, H, I, G, routes=list(range(T)))
+    check_routes(ro, ref, range(T))
+    assert torch.equal(out, ro)                       # weight 1: the combine is the route row
+    # every route dropped (ids out of range): zero rows, zero combine
+    bad = torch.full((T, 2), 5, dtype=torch.int32)
+    w2 = torch.full((T, 2), 0.5, dtype=torch.float32)
+    ro, out = cq.cq_moe_grouped_gemm(x.cuda(), bad.cuda(), w2.cuda(), layer, 1, H, I, G)
+    torch.cuda.synchronize()
+    assert cq.device_error() == (0, 0)
+    assert torch.all(ro == 0) and torch.all(out == 0)
+    # empty batch
+    ro, out = cq.cq_moe_grouped_gemm(x[:0].cuda(), ids[:0].cuda(), w[:0].cuda(), layer, 1, H,
+                                     I, G)
+    torch.cuda.synchronize()
+    assert ro.shape == (0, H) and out.shape == (0, H)
