@@ -569,6 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   long long prof_t = 0;
 
   if (tid == 0) {
+    griddep_launch_dependents();
     for (int s = 0; s < C::SW; ++s) {
       mbar_init(bar_wfull + 8 * s, 1);
       mbar_init(bar_wfree + 8 * s, kDecoders);
@@ -603,6 +604,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base =
       *reinterpret_cast<volatile uint32_t*>(gbase + (slot_tmem - base));
+  // programmatic dependent launch: the setup above overlapped the preceding
+  // grid; nothing written by it is read before this wait returns
+  griddep_wait();
 
   int num_tiles = p.num_tiles;
   if (p.grouped) num_tiles = ld_guarded(p.g_num_tiles);

@@ -75,7 +75,21 @@ static int launch_engine(const EngineParams& p, const CUtensorMap& map, const CU
       return CQ_ERR_CUDA;
     attr_set = true;
   }
-  engine_kernel<NT, TE><<<p.P, kThreads, C::SMEM, s>>>(p, map, wmap);
+  // programmatic dependent launch: this grid's setup (barriers, TMEM) may
+  // overlap the end of the preceding one; the kernel waits for it before
+  // reading any caller memory
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(p.P);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, engine_kernel<NT, TE>, p, map, wmap) != cudaSuccess)
+    return CQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
 }
 
