@@ -116,6 +116,13 @@ CQ_API int cq_decode(const uint8_t *packed, const float *scales, const uint16_t 
  *              counters that must be zero before the first call that uses
  *              the buffer; every completed call leaves them zero again.
  * Calls that share one workspace must not overlap on the GPU.
+ * Paths: M <= 2 runs the decode-sized GEMV kernel (no workspace: size 0);
+ * M >= 3 runs the tensor-core engine (128-row weight tiles, 16- to
+ * 192-token activation tiles, stream-K over the K slices, partial tiles
+ * summed in a fixed order).  Results are run-to-run deterministic.  Both
+ * kernels are launched with programmatic dependent launch: their setup may
+ * overlap the end of the preceding kernel in the stream, and they read no
+ * caller memory before that kernel has completed (stream order holds).
  */
 CQ_API size_t cq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int B, int G,
                               int epilogue);
