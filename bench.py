@@ -102,8 +102,11 @@ def dominant_kernel(name):
     if M <= 128:
         nt = 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
     else:
-        pad192, pad128 = -(-M // 192) * 192, -(-M // 128) * 128
-        nt = 192 if pad192 * 100 <= pad128 * (105 if B == 3 else 115) else 128
+        pad128 = -(-M // 128) * 128
+        if B == 3:
+            nt = 176 if -(-M // 176) * 176 * 100 <= pad128 * 105 else 128
+        else:
+            nt = 192 if -(-M // 192) * 192 * 100 <= pad128 * 115 else 128
     return f"engine_kernel<{nt},{64 if B == 3 else 16}>"
 
 

@@ -13,18 +13,24 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;   // 2 s per wait
 
 // Token-tile width.  Each token tile decodes the weights again, and up to
 // N = 192 the decode of a slice costs more than its MMAs, so wide problems
-// take 192-token tiles (the widest with two accumulator buffers in TMEM,
-// beside a ring of two decoded slices) unless the ragged last tile pads too
-// much against 128-token tiles: 15%, or 5% for W3, whose 64-entry pair
-// tables leave room for only two 192-token activation stages.  (256-token
-// tiles leave room for a single accumulator buffer: measured slower.)
+// take wide tiles with two accumulator buffers in TMEM (beside a ring of two
+// decoded slices): 192 tokens for W2/W4 and 176 for W3, whose 64-entry pair
+// tables leave room for only two 192-token activation stages but three of
+// 176 tokens -- unless the ragged last tile pads more than 15% (W3: 5%)
+// beyond 128-token tiles.  (256-token tiles leave room for a single
+// accumulator buffer: measured slower.)
 static int pick_nt(int64_t M, int B) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
   if (M <= 128) return 128;
-  const int64_t pad192 = (M + 191) / 192 * 192, pad128 = (M + 127) / 128 * 128;
-  return pad192 * 100 <= pad128 * (B == 3 ? 105 : 115) ? 192 : 128;
+  const int64_t pad128 = (M + 127) / 128 * 128;
+  if (B == 3) {
+    const int64_t pad176 = (M + 175) / 176 * 176;
+    return pad176 * 100 <= pad128 * 105 ? 176 : 128;
+  }
+  const int64_t pad192 = (M + 191) / 192 * 192;
+  return pad192 * 100 <= pad128 * 115 ? 192 : 128;
 }
 
 struct GemmPlan {
@@ -168,6 +174,7 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
     case 32: return launch_engine_te<32>(p, map, wmap, B, stream);
     case 64: return launch_engine_te<64>(p, map, wmap, B, stream);
     case 128: return launch_engine_te<128>(p, map, wmap, B, stream);
+    case 176: return launch_engine_te<176>(p, map, wmap, B, stream);
     default: return launch_engine_te<192>(p, map, wmap, B, stream);
   }
 }

@@ -132,6 +132,7 @@ GEMM_CASES = [
     # slices): two tiles with a ragged second one, one ragged tile under the
     # SwiGLU epilogue, and 128-token tiles where 192 would waste too much
     (380, 384,  1024, 3, 256, 0, 0, 0),
+    (350, 256,  1024, 3, 512, 0, 1, 1),      # W3: two 176-token tiles, ragged, SwiGLU
     (190, 256,  2048, 4, 512, 1, 1, 1),
     (256, 384,  2048, 4, 256, 0, 0, 0),
     (600, 256,  1024, 3, 128, 1, 1, 1),
