@@ -273,72 +273,63 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
 // decoder helpers
 // ---------------------------------------------------------------------------
 
-// Pair-table layout in shared memory: entry e of tile row i is the 32-bit
-// word at tbl + e*512 + 4*i, so the lookups of a warp always hit 32
-// distinct banks.  Entries:
-//   B=2: e = u0 | u1<<2 (16 entries)  ->  L[u0] | L[u1] << 16
-//   B=3: e = u0 | u1<<3 (64 entries)  ->  L[u0] | L[u1] << 16
-//   B=4: e = u        (16 entries)   ->  L[u]  | L[u]  << 16
-// with L_u = BF16(FP32(s sign(k) q(t))) the level of code u.  Levels are odd
-// in k (q(t) carries the sign), so only the positive side is evaluated in
-// FP64 and the negative codes flip the BF16 sign bit.
-template <int B, int HALF>
-__device__ __forceinline__ void build_table(uint32_t* tbl, int i, bool valid, float s,
-                                            uint32_t abw, int mode) {
+// The 2^B levels of one row's group (BF16 bits): q(t) in FP64, times s,
+// rounded once to FP32 and then to BF16.  Levels are odd in k (q(t) carries
+// the sign), so only the positive side is evaluated and the negative codes
+// flip the BF16 sign bit.
+template <int B>
+__device__ __forceinline__ void group_levels(bool valid, float s, uint32_t abw, int mode,
+                                             uint32_t (&L)[1 << B]) {
   constexpr int H = 1 << (B - 1);
-  uint32_t L[1 << B];
-  if (valid) {
-    const double a = static_cast<double>(__half2float(__ushort_as_half(abw & 0xFFFFu)));
-    const double b = static_cast<double>(__half2float(__ushort_as_half(abw >> 16)));
-    if (mode == CQ_GRID_MIDRISE) {
-      // codes H+j (j = 0..H-1) are the positive side, H-1-j their mirror
-#pragma unroll
-      for (int j = 0; j < H; ++j) {
-        const uint32_t m = bf16_bits(static_cast<float>(level_f64(H + j, B, 0, s, a, b)));
-        L[H + j] = m;
-        L[H - 1 - j] = m ^ 0x8000u;
-      }
-    } else {
-      // Kc = H-1; code Kc+m has |k| = m (m = 0..H), code Kc-m its mirror
-#pragma unroll
-      for (int m = 0; m <= H; ++m) {
-        const uint32_t v = bf16_bits(static_cast<float>(level_f64(H - 1 + m, B, 1, s, a, b)));
-        L[H - 1 + m] = v;
-        if (m >= 1 && m <= H - 1) L[H - 1 - m] = v ^ 0x8000u;
-      }
-    }
-  } else {
+  if (!valid) {
 #pragma unroll
     for (int u = 0; u < (1 << B); ++u) L[u] = 0u;
+    return;
   }
-  // this thread writes entries [half * E/2, (half + 1) * E/2)
-  if constexpr (B == 2) {
+  const double a = static_cast<double>(__half2float(__ushort_as_half(abw & 0xFFFFu)));
+  const double b = static_cast<double>(__half2float(__ushort_as_half(abw >> 16)));
+  if (mode == CQ_GRID_MIDRISE) {
+    // codes H+j (j = 0..H-1) are the positive side, H-1-j their mirror
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int e = HALF * 8 + k;
-      tbl[e * kRows + i] = L[e & 3] | (L[e >> 2] << 16);
-    }
-  } else if constexpr (B == 3) {
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const int e = HALF * 32 + k;
-      tbl[e * kRows + i] = L[e & 7] | (L[e >> 3] << 16);
+    for (int j = 0; j < H; ++j) {
+      const uint32_t m = bf16_bits(static_cast<float>(level_f64(H + j, B, 0, s, a, b)));
+      L[H + j] = m;
+      L[H - 1 - j] = m ^ 0x8000u;
     }
   } else {
+    // Kc = H-1; code Kc+m has |k| = m (m = 0..H), code Kc-m its mirror
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int e = HALF * 8 + k;
-      tbl[e * kRows + i] = L[e] | (L[e] << 16);
+    for (int m = 0; m <= H; ++m) {
+      const uint32_t v = bf16_bits(static_cast<float>(level_f64(H - 1 + m, B, 1, s, a, b)));
+      L[H - 1 + m] = v;
+      if (m >= 1 && m <= H - 1) L[H - 1 - m] = v ^ 0x8000u;
     }
   }
 }
 
-// Build the whole pair table of tile row i (every entry), levels as above.
+// Pair-table layout in shared memory: entry e of tile row i is the 32-bit
+// word at tbl + e*128 + i (words), so the lookups of a warp always hit 32
+// distinct banks.  Entries:
+//   B=2: e = u0 | u1<<2 (16 entries)  ->  L[u0] | L[u1] << 16
+//   B=3: e = u0 | u1<<3 (64 entries)  ->  L[u0] | L[u1] << 16
+//   B=4: e = u        (16 entries)   ->  L[u]  | L[u]  << 16
+// with L_u the level of code u.  One thread builds the whole table of its
+// row from one evaluation of the levels.
 template <int B>
 __device__ __forceinline__ void build_table_all(uint32_t* tbl, int i, bool valid, float s,
                                                 uint32_t abw, int mode) {
-  build_table<B, 0>(tbl, i, valid, s, abw, mode);
-  build_table<B, 1>(tbl, i, valid, s, abw, mode);
+  uint32_t L[1 << B];
+  group_levels<B>(valid, s, abw, mode, L);
+  if constexpr (B == 2) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) tbl[e * kRows + i] = L[e & 3] | (L[e >> 2] << 16);
+  } else if constexpr (B == 3) {
+#pragma unroll
+    for (int e = 0; e < 64; ++e) tbl[e * kRows + i] = L[e & 7] | (L[e >> 3] << 16);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) tbl[e * kRows + i] = L[e] | (L[e] << 16);
+  }
 }
 
 // Bits [sh, ...) of word w moved to bit 7 (the table's entry stride in words).
