@@ -8,15 +8,16 @@
 // sums the partial tiles in CTA order (deterministic) and applies the
 // epilogue.
 //
-// Warp roles (320 threads):
+// Warp roles (448 threads):
 //   warps 0-7  decoders: weight row i of the tile (TMEM lane i) belongs to
-//              thread i%32 of warps i/32 and i/32+4.  Per group the two
-//              build the row's BF16 pair table (two codes -> two levels,
-//              one 32-bit word per entry, the entries of all 128 rows
-//              interleaved so that every lookup of a warp hits 32 distinct
-//              banks) half each, then each turns its half of every 128-code
-//              slice into 32 BF16x2 words written to TMEM with tcgen05.st
-//              (the A operand of the MMA).
+//              thread i%32 of warps i/32 and i/32+4.  Warp q decodes the
+//              even slices and warp q+4 the odd ones, each slice whole
+//              (128 codes -> 64 BF16x2 words written to TMEM with
+//              tcgen05.st, the A operand of the MMA), each from its own BF16
+//              pair table per row (two codes -> two levels, one 32-bit word
+//              per entry, the entries of all 128 rows interleaved so that
+//              every lookup of a warp hits 32 distinct banks), so the two
+//              never wait for each other.
 //   warp 8     producer, two lanes with two rings of shared-memory stages:
 //              lane 0 loads, per 128-code slice, two 2-D TMA boxes of 64
 //              weight rows x 16*B bytes of packed codes (32-byte swizzle for
@@ -29,8 +30,9 @@
 //              TMEM (decoded weights) and B from shared memory
 //              (activations), FP32 accumulators in TMEM, double-buffered so
 //              the next tile's MMAs overlap the previous tile's epilogue
-//              (single-buffered at NT = 256, whose 256 accumulator columns
-//              fill the TMEM beside the A ring).
+//              (the ring of decoded slices shrinks from four to two at
+//              NT = 176/192 to make room; NT = 256 would leave room for
+//              only one accumulator buffer).
 //   warps 10-13 epilogue: tcgen05.ld of the accumulator, output conversion,
 //              SwiGLU, stream-K partials and their reduction.
 //
