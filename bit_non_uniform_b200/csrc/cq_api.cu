@@ -119,7 +119,7 @@ extern "C" int cq_pack(const uint8_t* codes, int64_t N, int64_t K, int B, uint8_
 extern "C" int cq_decode(const uint8_t* packed, const float* scales, const uint16_t* ab,
                          int64_t N, int64_t K, int B, int G, int grid_mode, int out_dtype,
                          void* W_out, void* stream) {
-  int st = validate_matrix(packed, scales, ab, N, K, B, G, grid_mode);
+  int st = validate_matrix(packed, scales, ab, N, K, B, G, grid_mode, 1, 8);
   if (st != CQ_OK) return st;
   if (!W_out) return CQ_ERR_INVALID_ARG;
   if (out_dtype != CQ_DTYPE_F32 && out_dtype != CQ_DTYPE_BF16) return CQ_ERR_INVALID_ARG;

@@ -15,11 +15,15 @@ inline bool aligned(const void* p, uintptr_t a) {
 }
 
 // Checks shared by every call that reads a packed CubicQuant matrix.
+// Bit widths: the GEMM paths take B in {2, 3, 4}; the format tools (pack,
+// decode) take 1..8 (the midtread grid needs B >= 2: Kc = 2^(B-1) - 1 > 0).
 inline int validate_matrix(const uint8_t* packed, const float* scales, const uint16_t* ab,
-                           int64_t N, int64_t K, int B, int G, int grid_mode) {
+                           int64_t N, int64_t K, int B, int G, int grid_mode, int b_min = 2,
+                           int b_max = 4) {
   if (N < 0 || K < 0 || G <= 0) return CQ_ERR_INVALID_ARG;
   if (grid_mode != CQ_GRID_MIDRISE && grid_mode != CQ_GRID_MIDTREAD) return CQ_ERR_INVALID_ARG;
-  if (B < 2 || B > 4) return CQ_ERR_UNSUPPORTED;
+  if (B < b_min || B > b_max) return CQ_ERR_UNSUPPORTED;
+  if (grid_mode == CQ_GRID_MIDTREAD && B < 2) return CQ_ERR_UNSUPPORTED;
   if (G % 128 != 0 || K % G != 0) return CQ_ERR_UNSUPPORTED;
   if (N * K == 0) return CQ_OK;
   if (!packed || !scales || !ab) return CQ_ERR_INVALID_ARG;

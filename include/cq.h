@@ -34,7 +34,9 @@
  *     NULL = legacy default stream) and returns a cq_status.  Arguments are
  *     validated on the host before anything is launched; on error nothing
  *     is launched and no output is touched.
- *   - Supported: B in {2,3,4}; G a multiple of 128; K a multiple of G;
+ *   - Supported: B in {2,3,4} for cq_gemm, cq_gemm_noalloc and the MoE
+ *     layer, B in 1..8 for cq_pack and cq_decode (midtread: 2..8);
+ *     G a multiple of 128; K a multiple of G;
  *     N >= 1; packed / x / y / workspace 16-byte aligned; scales and ab
  *     4-byte aligned.
  *   - The library allocates no memory.  Calls that need scratch take a
@@ -94,6 +96,7 @@ CQ_API int cq_pack(const uint8_t *codes, int64_t N, int64_t K, int B, uint8_t *p
  *             s*sign(k)*q(t) evaluated in FP64 and rounded once to FP32;
  *   out_dtype CQ_DTYPE_BF16: W_out bfloat16 [N][K], that FP32 value rounded
  *             to nearest-even BF16.
+ * B in 1..8 (midtread grid: 2..8); CQ_ERR_UNSUPPORTED otherwise.
  * [CQ] "CubicQuant 核心" (reconstruction); this is the parity tool, the GEMM
  * never materialises W ([CQ] "压缩权重必须“边解码、边计算”").
  */

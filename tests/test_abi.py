@@ -58,7 +58,8 @@ def test_pack_rejects_bad_arguments(lib):
 def test_decode_rejects_bad_arguments(lib):
     ok = (FAKE, FAKE, FAKE, 8, 512, 3, 128, 0, 0, FAKE, None)
     bad = [
-        ((FAKE, FAKE, FAKE, 8, 512, 5, 128, 0, 0, FAKE, None), 2),   # B = 5
+        ((FAKE, FAKE, FAKE, 8, 512, 9, 128, 0, 0, FAKE, None), 2),   # B = 9
+        ((FAKE, FAKE, FAKE, 8, 512, 1, 128, 1, 0, FAKE, None), 2),   # midtread needs B >= 2
         ((FAKE, FAKE, FAKE, 8, 512, 3, 100, 0, 0, FAKE, None), 2),   # G % 128
         ((FAKE, FAKE, FAKE, 8, 384, 3, 256, 0, 0, FAKE, None), 2),   # K % G
         ((FAKE, FAKE, FAKE, 8, 512, 3, 128, 7, 0, FAKE, None), 1),   # grid mode
@@ -80,7 +81,8 @@ def test_gemm_rejects_bad_arguments(lib):
         return lib.cq_gemm(a["x"], a["M"], a["packed"], a["scales"], a["ab"], a["N"], a["K"],
                            a["B"], a["G"], a["mode"], a["epi"], a["dt"], a["y"], a["ws"],
                            a["wsb"], a["s"])
-    assert call(B=1) == 2
+    assert call(B=1) == 2                     # the GEMM paths take B in {2, 3, 4}
+    assert call(B=5) == 2
     assert call(G=192) == 2
     assert call(K=640, G=256) == 2
     assert call(M=-1) == 1

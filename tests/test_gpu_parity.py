@@ -82,7 +82,7 @@ def test_generator_cpu_gpu_identical():
 # pack / decode
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("B", [2, 3, 4])
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("N,K", [(1, 128), (37, 256), (300, 1536)])
 def test_pack_bit_exact(cq, B, N, K):
     codes, _, _ = make_matrix(("pack", B, N), N, K, B, 128)
@@ -91,7 +91,10 @@ def test_pack_bit_exact(cq, B, N, K):
 
 
 @pytest.mark.parametrize("B,G,mode", [(2, 128, 0), (3, 512, 0), (4, 256, 0), (2, 128, 1),
-                                      (3, 256, 1), (4, 128, 1)])
+                                      (3, 256, 1), (4, 128, 1),
+                                      # the format tools also take 1 and 5..8 bits
+                                      (1, 128, 0), (5, 256, 0), (6, 128, 1), (7, 512, 0),
+                                      (8, 128, 0), (8, 256, 1)])
 def test_decode_within_one_ulp(cq, B, G, mode):
     N, K = 203, 1024
     codes, s, ab = make_matrix(("dec", B, G, mode), N, K, B, G, mode)

@@ -92,7 +92,11 @@ def _pack_by_bitstring(codes, B):
     return np.array(out, dtype=np.uint8)
 
 
-@pytest.mark.parametrize("B", [2, 3, 4])
+# widths of the format tools (pack, decode): 1..8; the GEMM paths use 2..4
+WIDTHS = [1, 2, 3, 4, 5, 6, 7, 8]
+
+
+@pytest.mark.parametrize("B", WIDTHS)
 def test_pack_exhaustive_small(B):
     K = 8 * (1 << B)             # every code value lands on every bit phase
     codes = np.array([[(k * 5 + r) % (1 << B) for k in range(K)] for r in range(3)],
@@ -102,9 +106,9 @@ def test_pack_exhaustive_small(B):
     assert np.array_equal(oracle.unpack(packed, K, B), codes)
 
 
-@pytest.mark.parametrize("B", [2, 3, 4])
+@pytest.mark.parametrize("B", WIDTHS)
 def test_pack_roundtrip_random(B):
-    codes = RNG.integers(0, 1 << B, size=(7, 384), dtype=np.uint8)
+    codes = RNG.integers(0, 1 << B, size=(7, 384), dtype=np.uint16).astype(np.uint8)
     assert np.array_equal(oracle.unpack(oracle.pack(codes, B), 384, B), codes)
 
 
@@ -125,11 +129,13 @@ def _coord_closed_form(u, B, mode):
     return u - Kc, Kc
 
 
-@pytest.mark.parametrize("B", [2, 3, 4])
+@pytest.mark.parametrize("B", WIDTHS)
 @pytest.mark.parametrize("mode", [oracle.MIDRISE, oracle.MIDTREAD])
 def test_basis_special_cases(B, mode):
     """q = t (a=1,b=0), q = t^2 (a=0,b=1), q = t^3 (a=0,b=0): each monomial
     of the cubic against the exact rational level sign(k)|k/Kc|^p."""
+    if mode == oracle.MIDTREAD and B < 2:
+        pytest.skip("the midtread grid needs B >= 2")
     s = 0.75
     ncodes = (1 << B) if mode == oracle.MIDRISE else (1 << B) - 1
     for (a, b, pw) in [(1.0, 0.0, 1), (0.0, 1.0, 2), (0.0, 0.0, 3)]:
@@ -140,7 +146,7 @@ def test_basis_special_cases(B, mode):
             assert lv[u] == pytest.approx(exact, rel=1e-15, abs=1e-300)
 
 
-@pytest.mark.parametrize("B", [2, 3, 4])
+@pytest.mark.parametrize("B", WIDTHS)
 def test_uniform_grid_midrise_is_linspace(B):
     """a = 1, b = 0 gives the symmetric uniform grid with 2^B levels spanning
     [-s, s] (section "CubicQuant 核心": the uniform integer grid is an exact
@@ -149,10 +155,10 @@ def test_uniform_grid_midrise_is_linspace(B):
     lv = oracle.levels(B, oracle.MIDRISE, s, _h(1.0), _h(0.0))
     assert np.allclose(lv, s * np.linspace(-1.0, 1.0, 1 << B), rtol=1e-14, atol=0)
     steps = np.diff(lv)
-    assert np.allclose(steps, steps[0], rtol=1e-12)
+    assert np.allclose(steps, steps[0], rtol=1e-11)
 
 
-@pytest.mark.parametrize("B", [2, 3, 4])
+@pytest.mark.parametrize("B", [2, 3, 4, 5, 6, 7, 8])
 def test_uniform_grid_midtread_is_signed_integer(B):
     s = 1.5
     Kc = (1 << (B - 1)) - 1
@@ -160,11 +166,13 @@ def test_uniform_grid_midtread_is_signed_integer(B):
     assert np.allclose(lv, s * np.arange(-Kc, Kc + 1) / Kc, rtol=1e-15)
 
 
-@pytest.mark.parametrize("B", [2, 3, 4])
+@pytest.mark.parametrize("B", WIDTHS)
 @pytest.mark.parametrize("mode", [oracle.MIDRISE, oracle.MIDTREAD])
 def test_exact_zero_and_endpoints(B, mode):
     """q(0) = 0 and q(1) = 1 exactly: the extreme codes decode to exactly
     -s and +s for every (a, b), and in midtread the middle code to 0."""
+    if mode == oracle.MIDTREAD and B < 2:
+        pytest.skip("the midtread grid needs B >= 2")
     for _ in range(200):
         a = float(np.float16(RNG.uniform(0.05, 2.5)))
         b = float(np.float16(RNG.uniform(-2, 2)))
