@@ -206,15 +206,17 @@ __device__ __forceinline__ int gv_div_spc(const GemvParams& p, int n) {
   return p.spc == 1 ? n : static_cast<int>(__umulhi(static_cast<uint32_t>(n), p.spc_magic));
 }
 
-// Sum of one output (entry e0 of column 0, row block rb) over the row
-// block's columns (group order) and their slice steps (in order), reading
-// the task partials of the CTA (task k of the CTA = its k-th quad-slice).
+// Part `sub` (0..3) of the sum of one output (entry e0 of column 0, row
+// block rb) over the row block's columns and their slice steps: the groups
+// gi = sub, sub + 4, ... in order, each group's slice steps in order
+// (task k of the CTA = its k-th quad-slice).  Four threads build the four
+// parts, which are then added in a fixed order.
 template <int NV, int MT>
-__device__ __forceinline__ float gv_rb_sum(const GemvParams& p, uint32_t slots, int rb, int e0,
-                                           int q_first) {
+__device__ __forceinline__ float gv_rb_sum_part(const GemvParams& p, uint32_t slots, int rb,
+                                                int e0, int q_first, int sub) {
   float v = 0.f;
-  int chi = rb * p.ng;
-  for (int gi = 0; gi < p.ng; ++gi, ++chi) {
+  for (int gi = sub; gi < p.ng; gi += 4) {
+    const int chi = rb * p.ng + gi;
     const int kb = ((chi >> 2) - q_first) * p.spc;
     const uint32_t src = slots + 4u * static_cast<uint32_t>((chi & 3) * (16 * MT) + e0);
     float t[4];
@@ -466,12 +468,21 @@ __device__ __forceinline__ void gemv_cta(const GemvParams& p, const CUtensorMap*
 
   // ------------------------------------------------------------------ phase D
   // out_f[rbl][r][m]: row slot r = 8 * item + g of row block rb_first + rbl
+  // four lanes per output, whole warps at a time (the shuffles need them)
   const int n_out = n_rbl * 16 * MT;
-  for (int o = tid; o < n_out; o += kGvThreads) {
-    const int m = o % MT;
-    const int r = (o / MT) & 15;
-    const int rb = rb_first + o / (16 * MT);
-    out_f[o] = gv_rb_sum<C::NV, MT>(p, slots, rb, r * MT + m, q_first);
+  for (int base4 = warp * 32; base4 < n_out * 4; base4 += kGvThreads) {
+    const int o4 = base4 + lane;
+    const int o = o4 >> 2;
+    float v = 0.f;
+    if (o < n_out) {
+      const int m = o % MT;
+      const int r = (o / MT) & 15;
+      const int rb = rb_first + o / (16 * MT);
+      v = gv_rb_sum_part<C::NV, MT>(p, slots, rb, r * MT + m, q_first, o4 & 3);
+    }
+    v += __shfl_xor_sync(0xffffffffu, v, 1);     // (part 0 + part 1), (part 2 + part 3)
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    if (o < n_out && (o4 & 3) == 0) out_f[o] = v;
   }
   __syncthreads();
   if (tid == 0) GV_STAMP(6);
