@@ -60,8 +60,8 @@ WORKLOADS = {
 # kernel and `traffic` is reported as null.
 KERNEL_SOURCES = ("cq_gemv.cuh", "cq_gemv_launch.cuh", "cq_device.cuh")
 TRAFFIC = {
-    "down_m1": {"kernel": "gemv_kernel<3,1>", "bytes": 8651776,
-                "sources_sha256": "9c0fd70674ae20b7b46b16200fe32c7edf8475c75be7cc9ec76340a56d490e7e"},
+    "down_m1": {"kernel": "gemv_kernel<3,1>", "bytes": 8652544,
+                "sources_sha256": "b8593820fe6ceb46c25dbb5d78b0eda2073dcceb0b9b846f2c38ba29ad423416"},
 }
 
 
