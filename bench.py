@@ -61,7 +61,7 @@ WORKLOADS = {
 KERNEL_SOURCES = ("cq_gemv.cuh", "cq_gemv_launch.cuh", "cq_device.cuh")
 TRAFFIC = {
     "down_m1": {"kernel": "gemv_kernel<3,1>", "bytes": 8652544,
-                "sources_sha256": "b8593820fe6ceb46c25dbb5d78b0eda2073dcceb0b9b846f2c38ba29ad423416"},
+                "sources_sha256": "253d37378681b15642e356880ad836961361511f58456029e3494acf30f3b2bb"},
 }
 
 

@@ -74,13 +74,8 @@ template <int NT, int TE>
 static int launch_engine(const EngineParams& p, const CUtensorMap& map, const CUtensorMap& wmap,
                          cudaStream_t s) {
   using C = EngineCfg<NT, TE>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(engine_kernel<NT, TE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM) != cudaSuccess)
-      return CQ_ERR_CUDA;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (!ensure_smem_limit(engine_kernel<NT, TE>, C::SMEM, smem_set)) return CQ_ERR_CUDA;
   // programmatic dependent launch: this grid's setup (barriers, TMEM) may
   // overlap the end of the preceding one; the kernel waits for it before
   // reading any caller memory

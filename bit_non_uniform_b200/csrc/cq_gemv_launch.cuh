@@ -66,13 +66,8 @@ static GvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int B, int G, int epilo
 
 template <int B, int MT>
 static int launch_gemv(const GemvParams& p, const CUtensorMap& wmap, int smem, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(gemv_kernel<B, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             227 * 1024) != cudaSuccess)
-      return CQ_ERR_CUDA;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (!ensure_smem_limit(gemv_kernel<B, MT>, 227 * 1024, smem_set)) return CQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(p.P);

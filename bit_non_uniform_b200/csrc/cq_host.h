@@ -2,6 +2,8 @@
 // shared by the libcq entry points.
 #pragma once
 
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -15,6 +17,23 @@ inline bool aligned(const void* p, uintptr_t a) {
 }
 
 // Checks shared by every call that reads a packed CubicQuant matrix.
+// Raise a kernel's dynamic shared-memory limit once per device: the
+// attribute belongs to the device's context, so a process that drives
+// several GPUs sets it on each (`done` holds one bit per device ordinal;
+// ordinals >= 64 set it on every call).
+template <typename Kernel>
+inline bool ensure_smem_limit(Kernel* kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const uint64_t bit = dev >= 0 && dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  if (bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
+
 // Bit widths: the GEMM paths take B in {2, 3, 4}; the format tools (pack,
 // decode) take 1..8 (the midtread grid needs B >= 2: Kc = 2^(B-1) - 1 > 0).
 inline int validate_matrix(const uint8_t* packed, const float* scales, const uint16_t* ab,

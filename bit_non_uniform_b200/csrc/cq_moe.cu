@@ -442,13 +442,11 @@ extern "C" int cq_moe_grouped_gemm(const uint16_t* tokens, int64_t T, const int3
 
   // 1. routing
   const size_t route_smem = (2 * static_cast<size_t>(E) + kRouteThreads + 1) * sizeof(int);
-  static bool route_attr = false;
-  if (!route_attr) {
-    if (cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (2 * kMaxExperts + kRouteThreads + 1) * sizeof(int)) != cudaSuccess)
-      return CQ_ERR_CUDA;
-    route_attr = true;
-  }
+  static std::atomic<uint64_t> route_smem_set{0};
+  if (!ensure_smem_limit(moe_route_kernel,
+                         static_cast<int>((2 * kMaxExperts + kRouteThreads + 1) * sizeof(int)),
+                         route_smem_set))
+    return CQ_ERR_CUDA;
   // decode-sized layers (few routes per expert) take the grouped GEMV path
   MoeGvParams gvp[2];
   const bool gv = moe_gemv_plan(m, T, k, E, H, I, G, grid_mode, sms, gvp);
@@ -481,13 +479,8 @@ extern "C" int cq_moe_grouped_gemm(const uint16_t* tokens, int64_t T, const int3
       q.out_rows = stage == 0 ? nullptr : perm;
       q.y_rows = m.R;
       q.R = m.R;
-      static bool attr = false;
-      if (!attr) {
-        if (cudaFuncSetAttribute(moe_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 227 * 1024) != cudaSuccess)
-          return CQ_ERR_CUDA;
-        attr = true;
-      }
+      static std::atomic<uint64_t> smem_set{0};
+      if (!ensure_smem_limit(moe_gemv_kernel<2>, 227 * 1024, smem_set)) return CQ_ERR_CUDA;
       moe_gemv_kernel<2><<<sms, kGvThreads, q.base.smem_bytes, s>>>(q);
       if (cudaGetLastError() != cudaSuccess) return CQ_ERR_CUDA;
     }
