@@ -119,6 +119,8 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
   if (!x || !y) return CQ_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(y, 16)) return CQ_ERR_UNSUPPORTED;
   if (M > (int64_t)1 << 24) return CQ_ERR_UNSUPPORTED;
+  // tile counts are int on the device: bound them by the narrowest token tile
+  if (((M + 15) / 16) * ((N + kRows - 1) / kRows) >= ((int64_t)1 << 31)) return CQ_ERR_UNSUPPORTED;
   const int sms = num_sms();
   if (sms <= 0) return CQ_ERR_CUDA;
   const GvPlan v = debug_skip ? GvPlan{} : plan_gemv(M, N, K, B, G, epilogue, sms);
@@ -177,8 +179,9 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int B, int G, int epilogue,
                            int sms) {
   if (M <= 0 || N <= 0 || K <= 0 || K % kSlice != 0 || G <= 0 || G % kSlice != 0 ||
-      K % G != 0)
-    return 0;
+      K % G != 0 || M > (int64_t)1 << 24 || N > (int64_t)1 << 30 ||
+      ((M + 15) / 16) * ((N + kRows - 1) / kRows) >= ((int64_t)1 << 31))
+    return 0;                                     // cq_gemm rejects these shapes
   size_t counters = 0, total = 0;
   gemm_scratch(M, N, K, B, G, epilogue, sms, &counters, &total);
   return total;

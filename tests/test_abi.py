@@ -90,6 +90,8 @@ def test_gemm_rejects_bad_arguments(lib):
     assert call(dt=2) == 1
     assert call(epi=1, N=200) == 2           # SwiGLU halves need N % 128 == 0
     assert call(M=0) == 0                     # empty problem is a no-op
+    assert call(M=(1 << 24) + 1) == 2         # beyond the supported token count
+    assert lib.cq_gemm_workspace_size((1 << 24) + 1, 256, 512, 3, 128, 0) == 0
     assert call(N=0) == 0
 
 
