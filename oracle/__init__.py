@@ -18,6 +18,12 @@ nearest level, the exact 1-D optimum as a lower bound, the clipped-uniform
 grid as an upper bound, consistency of its outputs) and, in midtread mode,
 by the article's W4 G128 NRMSE table.  The fitter's *midrise* NRMSE
 statistics: parity unpinned (the article prints none for that grid).
+
+The population analysis (``pop_*``, ``gap_recovery``: the error bound of
+"为什么只用两个形状参数？" evaluated on the Gaussian and Laplace densities) is
+pinned by quadrature, closed forms, the classical Lloyd-Max and optimum
+uniform quantizer tables, the Panter-Dite limit, and the article's W4..W8
+gap-recovery ranges (midtread grid) in ``tests/test_oracle_population.py``.
 """
 from __future__ import annotations
 
@@ -78,6 +84,13 @@ def _load():
                            P, P, P, P, P, i32]),
         "cqo_optimal_sse": (dbl, [P, i32, i32]),
         "cqo_num_threads": (i32, [i32]),
+        "cqo_pop_moments": (None, [i32, dbl, dbl, P]),
+        "cqo_pop_mse": (dbl, [i32, P, i32]),
+        "cqo_pop_lloyd_max": (dbl, [i32, i32, i32, dbl, P]),
+        "cqo_pop_shape": (None, [i32, dbl, dbl, P]),
+        "cqo_pop_monotone": (i32, [dbl, dbl]),
+        "cqo_pop_best_scale": (dbl, [i32, P, i32, P]),
+        "cqo_pop_cubic": (dbl, [i32, i32, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -350,3 +363,81 @@ def nearest(levels_sorted: np.ndarray, v: float, brute: bool = False) -> int:
 def optimal_sse(v: np.ndarray, nlev: int) -> float:
     v = np.ascontiguousarray(v, dtype=np.float64)
     return float(_load().cqo_optimal_sse(_ptr(v), len(v), nlev))
+
+
+# --------------------------------------------------------------------------
+# population analysis (the error bound of "为什么只用两个形状参数？")
+# --------------------------------------------------------------------------
+
+GAUSS = 0      # N(0, 1)
+LAPLACE = 1    # Laplace with unit variance
+
+
+def pop_moments(dist: int, a: float, b: float) -> np.ndarray:
+    """Integrals of x^j f(x) over [a, b], j = 0, 1, 2 (closed forms)."""
+    m = np.zeros(3)
+    _load().cqo_pop_moments(dist, float(a), float(b), _ptr(m))
+    return m
+
+
+def pop_mse(dist: int, levels: np.ndarray) -> float:
+    """MSE of the nearest-level quantizer with these levels on the density."""
+    lv = np.ascontiguousarray(np.sort(np.asarray(levels, dtype=np.float64)))
+    return float(_load().cqo_pop_mse(dist, _ptr(lv), len(lv)))
+
+
+def pop_lloyd_max(dist: int, n: int, max_iter: int = 100000, tol: float = 1e-13):
+    """n-level Lloyd-Max quantizer of the density: (MSE, ascending levels)."""
+    lv = np.zeros(n)
+    mse = _load().cqo_pop_lloyd_max(dist, n, max_iter, tol, _ptr(lv))
+    return float(mse), lv
+
+
+def pop_shape(n: int, a: float, b: float) -> np.ndarray:
+    """The n cubic levels on [-1, 1] (coordinate (2i - (n-1)) / (n-1))."""
+    out = np.zeros(n)
+    _load().cqo_pop_shape(n, float(a), float(b), _ptr(out))
+    return out
+
+
+def pop_monotone(a: float, b: float) -> bool:
+    return bool(_load().cqo_pop_monotone(float(a), float(b)))
+
+
+def pop_best_scale(dist: int, shape: np.ndarray):
+    """min over s of the MSE of s * shape: (MSE, s)."""
+    sh = np.ascontiguousarray(shape, dtype=np.float64)
+    s = ctypes.c_double()
+    mse = _load().cqo_pop_best_scale(dist, _ptr(sh), len(sh), ctypes.byref(s))
+    return float(mse), s.value
+
+
+def pop_uniform(dist: int, n: int):
+    """Best clipped uniform (INT) quantizer with n levels: (MSE, s)."""
+    return pop_best_scale(dist, pop_shape(n, 1.0, 0.0))
+
+
+def pop_cubic(dist: int, n: int):
+    """Best n-level cubic quantizer: (MSE, a, b, s)."""
+    a, b, s = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    mse = _load().cqo_pop_cubic(dist, n, ctypes.byref(a), ctypes.byref(b), ctypes.byref(s))
+    return float(mse), a.value, b.value, s.value
+
+
+def levels_of_width(B: int, mode: int) -> int:
+    """Distinct levels a B-bit code carries: 2^B on the midrise grid, 2^B - 1
+    on the midtread grid (its last code is unused)."""
+    return (1 << B) if mode == MIDRISE else (1 << B) - 1
+
+
+def gap_recovery(dist: int, B: int, mode: int) -> dict:
+    """Share of the best-INT / Lloyd-Max MSE gap that the best cubic closes,
+    (D_int - D_cubic) / (D_int - D_lloyd_max), all three with the same number
+    of levels, on the density itself (no sample)."""
+    n = levels_of_width(B, mode)
+    d_lm, _ = pop_lloyd_max(dist, n)
+    d_int, s_int = pop_uniform(dist, n)
+    d_cu, a, b, s = pop_cubic(dist, n)
+    return dict(n=n, lloyd_max=d_lm, int=d_int, int_s=s_int, cubic=d_cu, a=a, b=b, s=s,
+                recovered=(d_int - d_cu) / (d_int - d_lm))
+

@@ -30,6 +30,9 @@
  *   - groups are G consecutive elements along K inside one row; scales are
  *     float32 [N][K/G]; ab is fp16 [N][K/G][2] holding (a, b).
  *
+ * The end of the file evaluates [CQ two]'s error bound (Lloyd-Max <= Cubic
+ * <= best clipped INT) on the Gaussian and Laplace densities themselves.
+ *
  * Parity pins for every function are in tests/test_oracle_*.py.
  */
 #include <math.h>
@@ -541,4 +544,257 @@ double cqo_optimal_sse(const double *v_in, int n, int nlev)
 #undef DD
     free(D); free(S1); free(S2); free(v);
     return r;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Population analysis  [CQ two]: the error bound "Lloyd-Max <= Cubic <=    */
+/* best clipped INT" evaluated on a density instead of a finite sample, and */
+/* the share of the INT / Lloyd-Max gap that the cubic recovers.            */
+/* ------------------------------------------------------------------------ */
+
+#define CQO_DIST_GAUSS 0     /* N(0, 1) */
+#define CQO_DIST_LAPLACE 1   /* Laplace with unit variance: scale 1/sqrt(2) */
+
+static const double kLaplaceScale = 0.70710678118654752440;   /* 1/sqrt(2) */
+
+/* Upper-tail probability of N(0,1). */
+static double gauss_q(double x) { return 0.5 * erfc(x / 1.41421356237309504880); }
+static double gauss_pdf(double x) { return exp(-0.5 * x * x) * 0.39894228040143267794; }
+
+/*
+ * Partial moments m[j] = integral over [a, b] of x^j f(x), j = 0, 1, 2, for
+ * 0 <= a <= b (b may be +INFINITY), in closed form:
+ *   Gaussian:  m0 = Q(a) - Q(b),  m1 = pdf(a) - pdf(b),
+ *              m2 = m0 + a pdf(a) - b pdf(b)            (integration by parts)
+ *   Laplace (scale l): m0 = (e^{-a/l} - e^{-b/l}) / 2,
+ *              m1 = ((a + l) e^{-a/l} - (b + l) e^{-b/l}) / 2,
+ *              m2 = ((a^2 + 2 l a + 2 l^2) e^{-a/l} - (same at b)) / 2.
+ */
+static void half_moments(int dist, double a, double b, double m[3])
+{
+    int inf = isinf(b);
+    if (dist == CQO_DIST_GAUSS) {
+        double pa = gauss_pdf(a), pb = inf ? 0.0 : gauss_pdf(b);
+        m[0] = gauss_q(a) - (inf ? 0.0 : gauss_q(b));
+        m[1] = pa - pb;
+        m[2] = m[0] + a * pa - (inf ? 0.0 : b * pb);
+    } else {
+        double l = kLaplaceScale;
+        double ea = exp(-a / l), eb = inf ? 0.0 : exp(-b / l);
+        double bb = inf ? 0.0 : b;
+        m[0] = 0.5 * (ea - eb);
+        m[1] = 0.5 * ((a + l) * ea - (bb + l) * eb);
+        m[2] = 0.5 * ((a * a + 2 * l * a + 2 * l * l) * ea - (bb * bb + 2 * l * bb + 2 * l * l) * eb);
+    }
+}
+
+/* Partial moments over any interval a < b, using the symmetry of f. */
+void cqo_pop_moments(int dist, double a, double b, double *m)
+{
+    if (b <= 0) {
+        half_moments(dist, -b, -a, m);
+        m[1] = -m[1];
+    } else if (a >= 0) {
+        half_moments(dist, a, b, m);
+    } else {
+        double l[3], r[3];
+        half_moments(dist, 0.0, -a, l);
+        half_moments(dist, 0.0, b, r);
+        m[0] = l[0] + r[0];
+        m[1] = r[1] - l[1];
+        m[2] = l[2] + r[2];
+    }
+}
+
+/*
+ * Mean squared error of the nearest-level quantizer with the n levels lv
+ * (ascending) on the density: the decision thresholds are the midpoints of
+ * neighbouring levels, and each cell contributes the integral of
+ * (x - level)^2 f(x) = m2 - 2 level m1 + level^2 m0.
+ */
+double cqo_pop_mse(int dist, const double *lv, int n)
+{
+    double tot = 0.0;
+    for (int i = 0; i < n; i++) {
+        double lo = i == 0 ? -INFINITY : 0.5 * (lv[i - 1] + lv[i]);
+        double hi = i == n - 1 ? INFINITY : 0.5 * (lv[i] + lv[i + 1]);
+        double m[3];
+        cqo_pop_moments(dist, lo, hi, m);
+        tot += m[2] - 2.0 * lv[i] * m[1] + lv[i] * lv[i] * m[0];
+    }
+    return tot;
+}
+
+/* Inverse of an increasing function on the real line by bisection. */
+static double invert(double (*F)(double), double p)
+{
+    double lo = -60.0, hi = 60.0;
+    for (int it = 0; it < 200; it++) {
+        double mid = 0.5 * (lo + hi);
+        if (F(mid) < p) lo = mid; else hi = mid;
+    }
+    return 0.5 * (lo + hi);
+}
+
+/* CDFs of the point densities proportional to f^(1/3): N(0, 3) for the
+ * Gaussian, Laplace with three times the scale for the Laplace density. */
+static double cdf_gauss3(double x) { return 1.0 - gauss_q(x / 1.73205080756887729353); }
+static double cdf_laplace3(double x)
+{
+    double l = 3.0 * kLaplaceScale;
+    return x < 0 ? 0.5 * exp(x / l) : 1.0 - 0.5 * exp(-x / l);
+}
+
+/*
+ * Lloyd-Max quantizer with n levels (the free scalar codebook of [CQ two]'s
+ * bound) by Lloyd's iteration: thresholds at the midpoints of the levels,
+ * each level moved to the centroid m1/m0 of its cell, until no level moves
+ * by more than tol or max_iter sweeps.  Starts from the asymptotically
+ * optimal companding levels (quantiles of f^(1/3), Panter and Dite 1951).
+ * Writes the ascending levels to lv and returns their MSE.
+ */
+double cqo_pop_lloyd_max(int dist, int n, int max_iter, double tol, double *lv)
+{
+    double (*F)(double) = dist == CQO_DIST_GAUSS ? cdf_gauss3 : cdf_laplace3;
+    for (int i = 0; i < n; i++)
+        lv[i] = invert(F, (i + 0.5) / n);
+    double *nx = (double *)malloc(sizeof(double) * n);
+    for (int it = 0; it < max_iter; it++) {
+        double move = 0.0;
+        for (int i = 0; i < n; i++) {
+            double lo = i == 0 ? -INFINITY : 0.5 * (lv[i - 1] + lv[i]);
+            double hi = i == n - 1 ? INFINITY : 0.5 * (lv[i] + lv[i + 1]);
+            double m[3];
+            cqo_pop_moments(dist, lo, hi, m);
+            nx[i] = m[0] > 0 ? m[1] / m[0] : lv[i];
+            double d = fabs(nx[i] - lv[i]);
+            if (d > move) move = d;
+        }
+        memcpy(lv, nx, sizeof(double) * n);
+        if (move <= tol) break;
+    }
+    free(nx);
+    return cqo_pop_mse(dist, lv, n);
+}
+
+/*
+ * Level shape of an n-level cubic grid on [-1, 1]: code i has the signed
+ * coordinate (2i - (n-1)) / (n-1), i.e. t = |k| / Kc with Kc = (n-1)/2 --
+ * the midrise grid for n = 2^B and the midtread grid (without its unused
+ * code) for n = 2^B - 1 -- mapped through q  [CQ core].
+ */
+void cqo_pop_shape(int n, double a, double b, double *out)
+{
+    for (int i = 0; i < n; i++) {
+        double k = 2.0 * i - (n - 1);
+        double t = fabs(k) / (n - 1);
+        out[i] = (k > 0 ? 1.0 : (k < 0 ? -1.0 : 0.0)) * cqo_q(t, a, b);
+    }
+}
+
+/* Continuous counterpart of cqo_is_monotone: q'(t) > 0 on [0, 1]. */
+int cqo_pop_monotone(double a, double b)
+{
+    double c = 1.0 - a - b;
+    if (!(a > 0) || !(3.0 - 2.0 * a - b > 0))
+        return 0;
+    if (c > 0 && -b > 0 && -b < 3.0 * c && !(a - b * b / (3.0 * c) > 0))
+        return 0;
+    return 1;
+}
+
+/*
+ * min over the group scale s of the MSE of the levels s * shape (the
+ * clip threshold of a population quantizer is its scale): a scan of log s
+ * over [0.3, 40] in 64 steps, then golden-section search between the scan
+ * points around the best one.  Returns the MSE, writes s.
+ */
+double cqo_pop_best_scale(int dist, const double *shape, int n, double *s_out)
+{
+    double *lv = (double *)malloc(sizeof(double) * n);
+    const double l0 = log(0.3), l1 = log(40.0);
+    const int steps = 64;
+    double best = INFINITY;
+    int bi = 0;
+    for (int j = 0; j <= steps; j++) {
+        double s = exp(l0 + (l1 - l0) * j / steps);
+        for (int i = 0; i < n; i++) lv[i] = s * shape[i];
+        double e = cqo_pop_mse(dist, lv, n);
+        if (e < best) { best = e; bi = j; }
+    }
+    double lo = l0 + (l1 - l0) * (bi > 0 ? bi - 1 : 0) / steps;
+    double hi = l0 + (l1 - l0) * (bi < steps ? bi + 1 : steps) / steps;
+    const double gr = 0.61803398874989484820;
+    double x1 = hi - gr * (hi - lo), x2 = lo + gr * (hi - lo), f1, f2;
+    for (int i = 0; i < n; i++) lv[i] = exp(x1) * shape[i];
+    f1 = cqo_pop_mse(dist, lv, n);
+    for (int i = 0; i < n; i++) lv[i] = exp(x2) * shape[i];
+    f2 = cqo_pop_mse(dist, lv, n);
+    for (int it = 0; it < 60; it++) {
+        if (f1 < f2) {
+            hi = x2; x2 = x1; f2 = f1;
+            x1 = hi - gr * (hi - lo);
+            for (int i = 0; i < n; i++) lv[i] = exp(x1) * shape[i];
+            f1 = cqo_pop_mse(dist, lv, n);
+        } else {
+            lo = x1; x1 = x2; f1 = f2;
+            x2 = lo + gr * (hi - lo);
+            for (int i = 0; i < n; i++) lv[i] = exp(x2) * shape[i];
+            f2 = cqo_pop_mse(dist, lv, n);
+        }
+    }
+    double ls = f1 < f2 ? x1 : x2, e = f1 < f2 ? f1 : f2;
+    if (best < e) {                       /* the scan point itself was better */
+        e = best;
+        ls = l0 + (l1 - l0) * bi / steps;
+    }
+    free(lv);
+    if (s_out) *s_out = exp(ls);
+    return e;
+}
+
+static double cubic_cost(int dist, int n, double a, double b, double *shape, double *s)
+{
+    if (!cqo_pop_monotone(a, b)) return INFINITY;
+    cqo_pop_shape(n, a, b, shape);
+    return cqo_pop_best_scale(dist, shape, n, s);
+}
+
+/*
+ * Best n-level cubic quantizer of the density: min over monotone (a, b)
+ * and s of the MSE ([CQ fit]: search over monotone shape candidates jointly
+ * with the scale / clip).  A scan of a in [0.02, 2.92] and b in [-3, 3] with
+ * step 0.1 (plus the uniform point (1, 0)), then a pattern search around
+ * the best point: an 11 x 11 grid of step 0.02 that shrinks fourfold each
+ * round, eleven rounds.  Returns the MSE; writes a, b, s.
+ */
+double cqo_pop_cubic(int dist, int n, double *a_out, double *b_out, double *s_out)
+{
+    double *shape = (double *)malloc(sizeof(double) * n);
+    double s, ba = 1.0, bb = 0.0, bs = 0.0;
+    double best = cubic_cost(dist, n, 1.0, 0.0, shape, &bs);
+    for (int ia = 0; ia <= 29; ia++) {
+        for (int ib = 0; ib <= 60; ib++) {
+            double a = 0.02 + 0.1 * ia, b = -3.0 + 0.1 * ib;
+            double e = cubic_cost(dist, n, a, b, shape, &s);
+            if (e < best) { best = e; ba = a; bb = b; bs = s; }
+        }
+    }
+    double h = 0.02;
+    for (int round = 0; round < 11; round++) {
+        double ca = ba, cb = bb;
+        for (int ia = -5; ia <= 5; ia++) {
+            for (int ib = -5; ib <= 5; ib++) {
+                double a = ca + h * ia, b = cb + h * ib;
+                double e = cubic_cost(dist, n, a, b, shape, &s);
+                if (e < best) { best = e; ba = a; bb = b; bs = s; }
+            }
+        }
+        h *= 0.25;
+    }
+    free(shape);
+    if (a_out) *a_out = ba;
+    if (b_out) *b_out = bb;
+    if (s_out) *s_out = bs;
+    return best;
 }
