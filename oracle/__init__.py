@@ -19,6 +19,11 @@ grid as an upper bound, consistency of its outputs) and, in midtread mode,
 by the article's W4 G128 NRMSE table.  The fitter's *midrise* NRMSE
 statistics: parity unpinned (the article prints none for that grid).
 
+The Dynamic-A8 functions (``carrier``, ``quant_rows``, ``gemm_a8``, ``fit``
+with ``lam > 0``) are pinned in ``tests/test_oracle_a8.py`` by exact rational
+arithmetic, brute force on small cases, the special case where A8 equals the
+A16 product exactly, and the joint fit's invariants.
+
 The population analysis (``pop_*``, ``gap_recovery``: the error bound of
 "为什么只用两个形状参数？" evaluated on the Gaussian and Laplace densities) is
 pinned by quadrature, closed forms, the classical Lloyd-Max and optimum
@@ -82,7 +87,13 @@ def _load():
         "cqo_nearest_bruteforce": (i32, [P, i32, dbl]),
         "cqo_fit": (None, [P, i64, i32, i32, i32, P, i32, P, i32, P, i32, i32,
                            P, P, P, P, P, i32]),
+        "cqo_fit_joint": (None, [P, i64, i32, i32, i32, P, i32, P, i32, P, i32, i32, dbl,
+                                 P, P, P, P, P, P, i32]),
         "cqo_optimal_sse": (dbl, [P, i32, i32]),
+        "cqo_carrier": (i32, [i32, i32, i32, u16, u16]),
+        "cqo_carriers": (None, [i32, i32, u16, u16, P]),
+        "cqo_quant_rows": (None, [P, i64, i64, P, P]),
+        "cqo_gemm_a8": (None, [P, P, i64, P, P, P, i64, i64, i32, i32, i32, P, P]),
         "cqo_num_threads": (i32, [i32]),
         "cqo_pop_moments": (None, [i32, dbl, dbl, P]),
         "cqo_pop_mse": (dbl, [i32, P, i32]),
@@ -326,11 +337,13 @@ def default_grids():
 
 
 def fit(w: np.ndarray, G: int, B: int, mode=MIDRISE, uniform_only=False,
-        grids=None, nthreads=0):
-    """Fit every group of w (flattened, length multiple of G).
+        grids=None, nthreads=0, lam=0.0):
+    """Fit every group of w (flattened, length multiple of G), minimising
+    L_C + lam * L_A8 per group (lam = 0: the A16 fit; lam > 0: the A8
+    carrier correction of "一份 checkpoint，同时服务 A16 与 Dynamic A8").
 
     Returns dict(codes [ng][G] uint8, s [ng] f32, ab [ng][2] fp16 bits,
-    sse [ng], clipped [ng])."""
+    sse [ng] (L_C), sse_a8 [ng] (L_A8 of the same codes), clipped [ng])."""
     w = np.ascontiguousarray(np.asarray(w, dtype=np.float64).reshape(-1, G))
     ng = w.shape[0]
     a, b, alpha = grids if grids is not None else default_grids()
@@ -342,10 +355,11 @@ def fit(w: np.ndarray, G: int, B: int, mode=MIDRISE, uniform_only=False,
     ab = np.empty((ng, 2), dtype=np.uint16)
     sse = np.empty(ng, dtype=np.float64)
     clipped = np.empty(ng, dtype=np.int32)
-    _load().cqo_fit(_ptr(w), ng, G, B, mode, _ptr(a), len(a), _ptr(b), len(b),
-                    _ptr(alpha), len(alpha), int(uniform_only), _ptr(codes), _ptr(s),
-                    _ptr(ab), _ptr(sse), _ptr(clipped), nthreads)
-    return dict(codes=codes, s=s, ab=ab, sse=sse, clipped=clipped)
+    sse_a8 = np.empty(ng, dtype=np.float64)
+    _load().cqo_fit_joint(_ptr(w), ng, G, B, mode, _ptr(a), len(a), _ptr(b), len(b),
+                          _ptr(alpha), len(alpha), int(uniform_only), float(lam), _ptr(codes),
+                          _ptr(s), _ptr(ab), _ptr(sse), _ptr(clipped), _ptr(sse_a8), nthreads)
+    return dict(codes=codes, s=s, ab=ab, sse=sse, sse_a8=sse_a8, clipped=clipped)
 
 
 def nrmse(sse: np.ndarray, w: np.ndarray) -> float:
@@ -363,6 +377,48 @@ def nearest(levels_sorted: np.ndarray, v: float, brute: bool = False) -> int:
 def optimal_sse(v: np.ndarray, nlev: int) -> float:
     v = np.ascontiguousarray(v, dtype=np.float64)
     return float(_load().cqo_optimal_sse(_ptr(v), len(v), nlev))
+
+
+# --------------------------------------------------------------------------
+# Dynamic A8 ("一份 checkpoint，同时服务 A16 与 Dynamic A8")
+# --------------------------------------------------------------------------
+
+def carrier(u: int, B: int, mode: int, a_h: int, b_h: int) -> int:
+    """INT8 carrier of code u: RNE(127 sign(k) q(t)), saturated to +-127."""
+    return int(_load().cqo_carrier(u, B, mode, a_h, b_h))
+
+
+def carriers(B: int, mode: int, a_h: int, b_h: int) -> np.ndarray:
+    out = np.empty(1 << B, dtype=np.int8)
+    _load().cqo_carriers(B, mode, a_h, b_h, _ptr(out))
+    return out
+
+
+def quant_rows(x_bf16bits: np.ndarray):
+    """Per-row dynamic INT8 quantization of bf16 activations [M][K]:
+    returns (xq int8 [M][K], absmax f32 [M])."""
+    x = np.ascontiguousarray(x_bf16bits, dtype=np.uint16)
+    M, K = x.shape
+    xq = np.empty((M, K), dtype=np.int8)
+    absmax = np.empty(M, dtype=np.float32)
+    _load().cqo_quant_rows(_ptr(x), M, K, _ptr(xq), _ptr(absmax))
+    return xq, absmax
+
+
+def gemm_a8(xq, absmax, packed, scales, ab, N, K, B, G, mode=MIDRISE):
+    """Dynamic-A8 GEMM in FP64 from exact integer group sums: (y, bound),
+    both f64 [M][N]."""
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    absmax = np.ascontiguousarray(absmax, dtype=np.float32)
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    ab = np.ascontiguousarray(ab, dtype=np.uint16)
+    M = xq.shape[0]
+    y = np.empty((M, N), dtype=np.float64)
+    bound = np.empty((M, N), dtype=np.float64)
+    _load().cqo_gemm_a8(_ptr(xq), _ptr(absmax), M, _ptr(packed), _ptr(scales), _ptr(ab),
+                        N, K, B, G, mode, _ptr(y), _ptr(bound))
+    return y, bound
 
 
 # --------------------------------------------------------------------------

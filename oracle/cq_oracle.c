@@ -14,6 +14,7 @@
  *   [CQ bits]    "存储开销是透明的：B+64/G bit"          (storage identity)
  *   [CQ fit]     "从曲线到量化器：数据无关的组内拟合"     (group fitter)
  *   [CQ fused]   "压缩权重必须“边解码、边计算”"          (A16 execution)
+ *   [CQ a8]      "一份 checkpoint，同时服务 A16 与 Dynamic A8" (A8 mode)
  *
  * The article's displayed formulas were lost when the page was extracted;
  * the readings used here are:
@@ -28,7 +29,13 @@
  *     [k*B, k*B+B) of the row's byte stream, bit j in byte j/8 at bit j%8
  *     (the article only says "dense, contiguous"  [CQ two]);
  *   - groups are G consecutive elements along K inside one row; scales are
- *     float32 [N][K/G]; ab is fp16 [N][K/G][2] holding (a, b).
+ *     float32 [N][K/G]; ab is fp16 [N][K/G][2] holding (a, b);
+ *   - Dynamic A8 (its formulas were lost as well): the weight carrier of
+ *     code u is RNE(127 * sign(k) * q(t)) on the symmetric INT8 grid; each
+ *     activation row is quantized by its own absmax (x -> RNE(127 x /
+ *     absmax)); the integer dot product of a group is scaled by
+ *     (absmax / 127) * (s / 127); the joint fit minimises L_C + lambda *
+ *     L_A8 with the codes of the nearest continuous level.
  *
  * The end of the file evaluates [CQ two]'s error bound (Lloyd-Max <= Cubic
  * <= best clipped INT) on the Gaussian and Laplace densities themselves.
@@ -226,6 +233,108 @@ int cqo_is_monotone(uint16_t a_h, uint16_t b_h)
 }
 
 /* ------------------------------------------------------------------------ */
+/* Dynamic A8  [CQ a8]                                                       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * INT8 carrier of code u: the normalised level sign(k) q(t) placed on the
+ * symmetric INT8 grid, RNE(127 sign(k) q(t)) with q in FP64, saturated to
+ * [-127, 127] (only the midtread grid's unused code can leave that range).
+ * The carrier reconstruction of a weight is s * carrier / 127.
+ */
+int cqo_carrier(int u, int B, int mode, uint16_t a_h, uint16_t b_h)
+{
+    int sg;
+    double t;
+    cqo_coord(u, B, mode, &sg, &t);
+    double a = cqo_half_to_double(a_h);
+    double b = cqo_half_to_double(b_h);
+    double r = nearbyint(127.0 * (double)sg * cqo_q(t, a, b));  /* ties to even */
+    if (r > 127.0) r = 127.0;
+    if (r < -127.0) r = -127.0;
+    return (int)r;
+}
+
+/* All 2^B carriers of one group, in code order. */
+void cqo_carriers(int B, int mode, uint16_t a_h, uint16_t b_h, int8_t *out)
+{
+    for (int u = 0; u < (1 << B); u++)
+        out[u] = (int8_t)cqo_carrier(u, B, mode, a_h, b_h);
+}
+
+/*
+ * Dynamic per-row INT8 quantization of bf16 activations x [M][K]: absmax =
+ * max |x| of the row; inv = 127 / absmax and every product x * inv rounded
+ * to FP32, then to the nearest integer (ties to even), saturated to
+ * [-127, 127].  These decisions are taken in FP32, the precision of a GPU
+ * kernel taking them.  A zero row gives absmax 0 and all-zero codes.
+ */
+void cqo_quant_rows(const uint16_t *x, int64_t M, int64_t K, int8_t *xq, float *absmax)
+{
+    for (int64_t m = 0; m < M; m++) {
+        float mx = 0.0f;
+        for (int64_t k = 0; k < K; k++) {
+            float v = (float)cqo_bf16_to_double(x[m * K + k]);
+            if (fabsf(v) > mx) mx = fabsf(v);
+        }
+        absmax[m] = mx;
+        float inv = mx > 0.0f ? 127.0f / mx : 0.0f;
+        for (int64_t k = 0; k < K; k++) {
+            float v = (float)cqo_bf16_to_double(x[m * K + k]);
+            float p = v * inv;
+            float r = nearbyintf(p);
+            if (r > 127.0f) r = 127.0f;
+            if (r < -127.0f) r = -127.0f;
+            xq[m * K + k] = (int8_t)r;
+        }
+    }
+}
+
+/*
+ * Dynamic-A8 GEMM: for every (m, n) and group g the exact integer dot
+ * product acc = sum over the group of xq[m][k] * carrier(u[n][k]), then
+ * the group scaling y[m][n] = sum_g (absmax[m] / 127) (s[n][g] / 127) acc,
+ * here in FP64 with the groups in order.  bound[m][n] (may be NULL) is the
+ * same sum over |xq * carrier|: the scale of the tolerance.
+ */
+void cqo_gemm_a8(const int8_t *xq, const float *absmax, int64_t M, const uint8_t *packed,
+                 const float *scales, const uint16_t *ab, int64_t N, int64_t K, int B, int G,
+                 int mode, double *y, double *bound)
+{
+    int64_t ng = K / G, rb = K * B / 8;
+    uint8_t *codes = (uint8_t *)malloc((size_t)K);
+    int8_t *car = (int8_t *)malloc((size_t)K);
+    int8_t tab[256];
+    for (int64_t n = 0; n < N; n++) {
+        cqo_unpack(packed + n * rb, 1, K, B, codes);
+        for (int64_t g = 0; g < ng; g++) {
+            cqo_carriers(B, mode, ab[(n * ng + g) * 2 + 0], ab[(n * ng + g) * 2 + 1], tab);
+            for (int64_t k = g * G; k < (g + 1) * G; k++)
+                car[k] = tab[codes[k]];
+        }
+        for (int64_t m = 0; m < M; m++) {
+            double acc_y = 0.0, acc_b = 0.0;
+            double sx = (double)absmax[m] / 127.0;
+            for (int64_t g = 0; g < ng; g++) {
+                int64_t acc = 0, aabs = 0;
+                for (int64_t k = g * G; k < (g + 1) * G; k++) {
+                    int64_t p = (int64_t)xq[m * K + k] * (int64_t)car[k];
+                    acc += p;
+                    aabs += p < 0 ? -p : p;
+                }
+                double f = sx * ((double)scales[n * ng + g] / 127.0);
+                acc_y += f * (double)acc;
+                acc_b += fabs(f) * (double)aabs;
+            }
+            y[m * N + n] = acc_y;
+            if (bound) bound[m * N + n] = acc_b;
+        }
+    }
+    free(codes);
+    free(car);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Decode  [CQ core] + [CQ fused]                                            */
 /* ------------------------------------------------------------------------ */
 
@@ -366,6 +475,7 @@ typedef struct {
     int na, nb, nalpha;
     const double *a_grid, *b_grid, *alpha_grid;
     int uniform_only;          /* 1: only (a,b) = (1,0)  -> optimal clipped INT */
+    double lambda;             /* weight of the carrier error in the objective */
 } fit_cfg;
 
 /* Number of codes a grid mode uses: 2^B (midrise) or 2^B - 1 (midtread). */
@@ -374,23 +484,36 @@ static int used_levels(int B, int mode)
     return mode == CQO_MIDRISE ? (1 << B) : (1 << B) - 1;
 }
 
-/* SSE of group w[G] under (s, a_h, b_h); codes written when out != NULL. */
+/*
+ * SSE of group w[G] under (s, a_h, b_h) with every weight on its nearest
+ * continuous level; codes written when codes_out != NULL.  When sse_a8 is
+ * not NULL it receives the carrier error of the same codes, the sum of
+ * (w - s * carrier(u) / 127)^2  [CQ a8].
+ */
 static double group_sse(const double *w, int G, int B, int mode, float s,
-                        uint16_t a_h, uint16_t b_h, uint8_t *codes_out, int *clipped)
+                        uint16_t a_h, uint16_t b_h, uint8_t *codes_out, int *clipped,
+                        double *sse_a8)
 {
     double lv[256];
+    int8_t car[256];
     int nl = used_levels(B, mode);
     cqo_levels(B, mode, s, a_h, b_h, lv);
-    double sse = 0.0;
+    if (sse_a8) cqo_carriers(B, mode, a_h, b_h, car);
+    double sse = 0.0, sse8 = 0.0;
     int clip = 0;
     for (int i = 0; i < G; i++) {
         int u = cqo_nearest(lv, nl, w[i]);
         double e = w[i] - lv[u];
         sse += e * e;
+        if (sse_a8) {
+            double e8 = w[i] - (double)s * (double)car[u] / 127.0;
+            sse8 += e8 * e8;
+        }
         if (fabs(w[i]) > (double)s) clip++;
         if (codes_out) codes_out[i] = (uint8_t)u;
     }
     if (clipped) *clipped = clip;
+    if (sse_a8) *sse_a8 = sse8;
     return sse;
 }
 
@@ -403,14 +526,17 @@ static double group_sse(const double *w, int G, int B, int mode, float s,
  *   (4) assign every weight to its nearest reconstruction level;
  *   (5) cast a, b to FP16 and keep s in FP32, then recompute the codes and
  *       the error with the stored values.
- * The objective is the group's squared error.  Ties keep the earliest
- * candidate in enumeration order: (1,0) first, then the (a,b) grid in order,
- * and for each (a,b) alpha ascending.
- * Outputs: codes[G], s, a_h, b_h; return value = SSE with stored values.
+ * The objective is the group's squared error L_C, plus lambda times the
+ * carrier error L_A8 of the same codes when lambda > 0 (the A8 carrier
+ * correction of [CQ a8]).  Ties keep the earliest candidate in enumeration
+ * order: (1,0) first, then the (a,b) grid in order, and for each (a,b)
+ * alpha ascending.
+ * Outputs: codes[G], s, a_h, b_h, the carrier error (sse_a8, may be NULL);
+ * return value = L_C with the stored values.
  */
 static double fit_group(const double *w, int G, int B, int mode, const fit_cfg *cfg,
                         uint8_t *codes, float *s_out, uint16_t *a_out, uint16_t *b_out,
-                        int *clipped)
+                        int *clipped, double *sse_a8)
 {
     double mx = 0.0;
     for (int i = 0; i < G; i++)
@@ -419,8 +545,9 @@ static double fit_group(const double *w, int G, int B, int mode, const fit_cfg *
         *s_out = 0.0f;
         *a_out = cqo_double_to_half(1.0);
         *b_out = cqo_double_to_half(0.0);
-        return group_sse(w, G, B, mode, 0.0f, *a_out, *b_out, codes, clipped);
+        return group_sse(w, G, B, mode, 0.0f, *a_out, *b_out, codes, clipped, sse_a8);
     }
+    const int joint = cfg->lambda > 0.0;
     double best = INFINITY;
     double best_a = 1.0, best_b = 0.0;
     float best_s = (float)mx;
@@ -437,7 +564,9 @@ static double fit_group(const double *w, int G, int B, int mode, const fit_cfg *
         if (!cqo_is_monotone(a_h, b_h)) continue;
         for (int ia = 0; ia < cfg->nalpha; ia++) {
             float s = (float)(cfg->alpha_grid[ia] * mx);
-            double e = group_sse(w, G, B, mode, s, a_h, b_h, NULL, NULL);
+            double e8 = 0.0;
+            double e = group_sse(w, G, B, mode, s, a_h, b_h, NULL, NULL, joint ? &e8 : NULL);
+            if (joint) e += cfg->lambda * e8;
             if (e < best) { best = e; best_a = a; best_b = b; best_s = s; }
         }
     }
@@ -445,13 +574,13 @@ static double fit_group(const double *w, int G, int B, int mode, const fit_cfg *
     *a_out = cqo_double_to_half(best_a);
     *b_out = cqo_double_to_half(best_b);
     *s_out = best_s;
-    return group_sse(w, G, B, mode, best_s, *a_out, *b_out, codes, clipped);
+    return group_sse(w, G, B, mode, best_s, *a_out, *b_out, codes, clipped, sse_a8);
 }
 
 typedef struct {
     const double *w; int64_t ngroups; int G, B, mode;
     const fit_cfg *cfg;
-    uint8_t *codes; float *s; uint16_t *ab; double *sse; int32_t *clipped;
+    uint8_t *codes; float *s; uint16_t *ab; double *sse; int32_t *clipped; double *sse_a8;
     int64_t g0, g1;
 } fit_job;
 
@@ -462,7 +591,7 @@ static void *fit_worker(void *p)
         int clip = 0;
         double e = fit_group(j->w + g * j->G, j->G, j->B, j->mode, j->cfg,
                              j->codes + g * j->G, &j->s[g], &j->ab[2 * g],
-                             &j->ab[2 * g + 1], &clip);
+                             &j->ab[2 * g + 1], &clip, j->sse_a8 ? &j->sse_a8[g] : NULL);
         j->sse[g] = e;
         j->clipped[g] = clip;
     }
@@ -470,23 +599,25 @@ static void *fit_worker(void *p)
 }
 
 /*
- * Fit ngroups independent groups of G weights (w is [ngroups][G]).
+ * Fit ngroups independent groups of G weights (w is [ngroups][G]) with the
+ * objective L_C + lambda * L_A8 (lambda = 0: the A16 fit).
  * Outputs per group: codes [ngroups][G], s [ngroups], ab [ngroups][2] (fp16
- * bits), sse [ngroups], clipped [ngroups] (count of |w| > s).
+ * bits), sse [ngroups] (L_C), clipped [ngroups] (count of |w| > s), and
+ * sse_a8 [ngroups] (L_A8, may be NULL).
  */
-void cqo_fit(const double *w, int64_t ngroups, int G, int B, int mode,
-             const double *a_grid, int na, const double *b_grid, int nb,
-             const double *alpha_grid, int nalpha, int uniform_only,
-             uint8_t *codes, float *s, uint16_t *ab, double *sse, int32_t *clipped,
-             int nthreads)
+void cqo_fit_joint(const double *w, int64_t ngroups, int G, int B, int mode,
+                   const double *a_grid, int na, const double *b_grid, int nb,
+                   const double *alpha_grid, int nalpha, int uniform_only, double lambda,
+                   uint8_t *codes, float *s, uint16_t *ab, double *sse, int32_t *clipped,
+                   double *sse_a8, int nthreads)
 {
-    fit_cfg cfg = {na, nb, nalpha, a_grid, b_grid, alpha_grid, uniform_only};
+    fit_cfg cfg = {na, nb, nalpha, a_grid, b_grid, alpha_grid, uniform_only, lambda};
     int T = cqo_num_threads(nthreads);
     if (T > ngroups) T = (int)(ngroups > 0 ? ngroups : 1);
     pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * T);
     fit_job *jobs = (fit_job *)malloc(sizeof(fit_job) * T);
     for (int i = 0; i < T; i++) {
-        fit_job j = {w, ngroups, G, B, mode, &cfg, codes, s, ab, sse, clipped,
+        fit_job j = {w, ngroups, G, B, mode, &cfg, codes, s, ab, sse, clipped, sse_a8,
                      ngroups * i / T, ngroups * (i + 1) / T};
         jobs[i] = j;
         pthread_create(&th[i], NULL, fit_worker, &jobs[i]);
@@ -495,6 +626,17 @@ void cqo_fit(const double *w, int64_t ngroups, int G, int B, int mode,
         pthread_join(th[i], NULL);
     free(th);
     free(jobs);
+}
+
+/* The A16 fit: cqo_fit_joint with lambda = 0. */
+void cqo_fit(const double *w, int64_t ngroups, int G, int B, int mode,
+             const double *a_grid, int na, const double *b_grid, int nb,
+             const double *alpha_grid, int nalpha, int uniform_only,
+             uint8_t *codes, float *s, uint16_t *ab, double *sse, int32_t *clipped,
+             int nthreads)
+{
+    cqo_fit_joint(w, ngroups, G, B, mode, a_grid, na, b_grid, nb, alpha_grid, nalpha,
+                  uniform_only, 0.0, codes, s, ab, sse, clipped, NULL, nthreads);
 }
 
 /*
