@@ -165,3 +165,29 @@ def test_experts_must_split_evenly():
     assert experts_per_rank(896, 8) == 112
     with pytest.raises(ValueError):
         experts_per_rank(10, 4)
+
+
+def test_libcq_compute_calls_the_grouped_gemm(monkeypatch):
+    # the product's expert compute hands the received rows to cq_moe_grouped_gemm with
+    # the rank's own expert count, no per-route output and the combine on; a rank that
+    # receives nothing makes no call
+    import bit_non_uniform_b200 as cq
+    from bit_non_uniform_b200.ep import libcq_compute
+    seen = []
+
+    def fake(tokens, ids, w, layer, E, H_, I_, G_, mode, out_dtype, route_out, combine):
+        seen.append((tokens.shape, ids.shape, w.shape, layer, E, H_, I_, G_, mode, out_dtype,
+                     route_out, combine))
+        return None, torch.full((tokens.shape[0], H_), 2.0)
+
+    monkeypatch.setattr(cq, "cq_moe_grouped_gemm", fake)
+    run = libcq_compute("layer-table", 4, H, I, G, mode=1)
+    x = torch.zeros((3, H), dtype=torch.bfloat16)
+    ids = torch.zeros((3, K_TOP), dtype=torch.int32)
+    w = torch.zeros((3, K_TOP), dtype=torch.float32)
+    out = run(x, ids, w)
+    assert torch.equal(out, torch.full((3, H), 2.0))
+    assert seen == [((3, H), (3, K_TOP), (3, K_TOP), "layer-table", 4, H, I, G, 1, cq.F32,
+                     None, True)]
+    empty = run(x[:0], ids[:0], w[:0])
+    assert empty.shape == (0, H) and empty.dtype == torch.float32 and len(seen) == 1
