@@ -202,3 +202,23 @@ def test_moe_degenerate_layers(cq):
                                      I, G)
     torch.cuda.synchronize()
     assert ro.shape == (0, H) and out.shape == (0, H)
+
+
+def test_expert_parallel_single_rank_is_the_grouped_gemm(cq):
+    """The expert-parallel layer on one rank (no process group) hands every
+    token row, in order, with its ids unchanged, to the same grouped GEMM:
+    the output is bit-identical to calling cq_moe_grouped_gemm directly."""
+    from bit_non_uniform_b200.ep import MoeExpertParallel, libcq_compute
+    H, I, E, T, k, G = 512, 256, 8, 37, 2, 128
+    tag = ("ep1", H, E, T)
+    Bs = [(2, 3, 4)[e % 3] for e in range(E)]
+    experts = [expert_gpu(cq, tag, e, Bs[e], H, I, G) for e in range(E)]
+    layer = cq.moe_prepare_layer(experts, H, I, G)
+    x = synthetic.activations(T + 9, T, H).cuda()
+    ids, w = synthetic.routing_uniform(T + 9, T, E, k)
+    ids, w = ids.cuda(), w.cuda()
+    _, direct = cq.cq_moe_grouped_gemm(x, ids, w, layer, E, H, I, G)
+    got = MoeExpertParallel(E, H, libcq_compute(layer, E, H, I, G)).forward(x, ids, w)
+    torch.cuda.synchronize()
+    assert cq.device_error() == (0, 0)
+    assert got.dtype == torch.float32 and torch.equal(got, direct)
