@@ -29,7 +29,8 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "cq.h")]
+    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [
+        os.path.join(INCLUDE, h) for h in ("cq.h", "cq_hooks.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include "cq.h"
+#include "cq_hooks.h"
 #include "cq_engine.cuh"
 #include "cq_gemv_launch.cuh"
 #include "cq_host.h"
@@ -103,11 +104,11 @@ static int launch_engine_te(const EngineParams& p, const CUtensorMap& map,
   return launch_engine<NT, 16>(p, map, wmap, s);
 }
 
-int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* scales,
-              const uint16_t* ab, int64_t N, int64_t K, int B, int G, int grid_mode,
-              int epilogue, int out_dtype, void* y, void* workspace, size_t ws_bytes,
-              cudaStream_t stream, uint64_t timeout_ns, int debug_skip,
-              uint64_t* trace = nullptr) {
+// Every argument and shape check of cq_gemm except the workspace: a call that
+// passes launches nothing unless the problem is empty (M == 0 or N == 0).
+static int validate_gemm(const uint16_t* x, int64_t M, const uint8_t* packed,
+                         const float* scales, const uint16_t* ab, int64_t N, int64_t K, int B,
+                         int G, int grid_mode, int epilogue, int out_dtype, const void* y) {
   int st = validate_matrix(packed, scales, ab, N, K, B, G, grid_mode);
   if (st != CQ_OK) return st;
   if (M < 0) return CQ_ERR_INVALID_ARG;
@@ -121,6 +122,18 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
   if (M > (int64_t)1 << 24) return CQ_ERR_UNSUPPORTED;
   // tile counts are int on the device: bound them by the narrowest token tile
   if (((M + 15) / 16) * ((N + kRows - 1) / kRows) >= ((int64_t)1 << 31)) return CQ_ERR_UNSUPPORTED;
+  return CQ_OK;
+}
+
+int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* scales,
+              const uint16_t* ab, int64_t N, int64_t K, int B, int G, int grid_mode,
+              int epilogue, int out_dtype, void* y, void* workspace, size_t ws_bytes,
+              cudaStream_t stream, uint64_t timeout_ns, int debug_skip,
+              uint64_t* trace = nullptr) {
+  int st = validate_gemm(x, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype,
+                         y);
+  if (st != CQ_OK) return st;
+  if (M == 0 || N == 0) return CQ_OK;
   const int sms = num_sms();
   if (sms <= 0) return CQ_ERR_CUDA;
   const GvPlan v = debug_skip ? GvPlan{} : plan_gemv(M, N, K, B, G, epilogue, sms);
@@ -206,9 +219,8 @@ extern "C" int cq_gemm(const uint16_t* x, int64_t M, const uint8_t* packed, cons
                    workspace, ws_bytes, static_cast<cudaStream_t>(stream), kDefaultTimeoutNs, 0);
 }
 
-// Profiling hook (not part of the public header): cq_gemm that also writes
-// per-CTA event timestamps to trace ([grid][64] uint64, device memory, at
-// least cq_gemm_workspace_size-independent 148*64 entries).
+// Profiling hook (declared in cq_hooks.h): cq_gemm that also writes per-CTA
+// event timestamps to trace ([grid][64] uint64 words of device memory).
 extern "C" CQ_API int cq_trace_gemm(const uint16_t* x, int64_t M, const uint8_t* packed,
                                     const float* scales, const uint16_t* ab, int64_t N,
                                     int64_t K, int B, int G, int epilogue, void* y,
@@ -219,10 +231,9 @@ extern "C" CQ_API int cq_trace_gemm(const uint16_t* x, int64_t M, const uint8_t*
                    kDefaultTimeoutNs, 0, trace);
 }
 
-// Test hook (not part of the public header): run cq_gemm with a chosen wait
-// limit and, optionally, with the first stage load withheld so that the
-// bounded waits run out; the caller then reads CQ_ERR_TIMEOUT from
-// cq_get_device_error().
+// Test hook (declared in cq_hooks.h): cq_gemm with a chosen wait limit and,
+// optionally, with the first stage loads withheld so that the bounded waits
+// run out; the caller then reads CQ_ERR_TIMEOUT from cq_get_device_error().
 extern "C" CQ_API int cq_test_gemm_bounded(const uint16_t* x, int64_t M, const uint8_t* packed,
                                     const float* scales, const uint16_t* ab, int64_t N, int64_t K,
                                     int B, int G, void* y, void* workspace, size_t ws_bytes,

@@ -146,11 +146,15 @@ CQ_API int cq_gemm(const uint16_t *x, int64_t M, const uint8_t *packed, const fl
  *   library holds it until the process exits), enough for any M <= 16 on a
  *   148-SM B200; a problem that needs more returns CQ_ERR_WORKSPACE.
  *   The first call on a device looks up that array's device address (a CUDA
- *   runtime query) and caches it; make that first call before any stream
- *   capture.  Every call shares the one array: calls that overlap on the GPU
- *   (other streams, other host threads) race and must not be issued.
- *   Each call clears the array's tile counters with cudaMemsetAsync on
- *   `stream`; it calls no allocating routine.
+ *   runtime query, which also loads libcq's device code there) and caches
+ *   it with the device's context; make that first call before any stream
+ *   capture.  After a cudaDeviceReset the device has a new context and the
+ *   next call looks the address up again (again: not inside a capture).
+ *   Every call shares the one array: calls that overlap on the GPU (other
+ *   streams, other host threads) race and must not be issued.  All argument
+ *   checks run before anything is queued; a call that passes them clears
+ *   the array's tile counters with cudaMemsetAsync on `stream`.  It calls
+ *   no allocating or freeing routine.
  */
 CQ_API int cq_gemm_noalloc(const uint16_t *x, int64_t M, const uint8_t *packed,
                            const float *scales, const uint16_t *ab, int64_t N, int64_t K, int B,

@@ -10,8 +10,8 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _declared_symbols():
-    with open(os.path.join(ROOT, "include", "cq.h")) as f:
+def _declared_symbols(header="cq.h"):
+    with open(os.path.join(ROOT, "include", header)) as f:
         text = f.read()
     return sorted(set(re.findall(r"^\s*(?:CQ_API\s+)?(?:int|size_t|const char\s*\*)\s*(cq_\w+)\s*\(", text,
                                  re.M)))
@@ -35,6 +35,13 @@ def test_header_declares_the_boundary():
 
 def test_library_exports_every_declared_symbol(lib):
     for s in _declared_symbols():
+        assert hasattr(lib, s), s
+
+
+def test_hooks_are_declared_and_exported(lib):
+    hooks = _declared_symbols("cq_hooks.h")
+    assert hooks == ["cq_test_gemm_bounded", "cq_trace_gemm"]
+    for s in hooks:
         assert hasattr(lib, s), s
 
 
@@ -93,6 +100,31 @@ def test_gemm_rejects_bad_arguments(lib):
     assert call(M=(1 << 24) + 1) == 2         # beyond the supported token count
     assert lib.cq_gemm_workspace_size((1 << 24) + 1, 256, 512, 3, 128, 0) == 0
     assert call(N=0) == 0
+
+
+def test_gemm_noalloc_rejects_bad_arguments_before_touching_the_gpu(lib):
+    """Every check runs before the fixed array is looked up or cleared: on a
+    machine without a GPU these calls return their status without a CUDA
+    call failing first."""
+    f = lib.cq_gemm_noalloc
+    P = ctypes.c_void_p
+    f.argtypes = [P, ctypes.c_int64, P, P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
+
+    def call(**kw):
+        a = dict(x=FAKE, M=4, packed=FAKE, scales=FAKE, ab=FAKE, N=256, K=512, B=3, G=128,
+                 mode=0, epi=0, dt=0, y=FAKE, s=None)
+        a.update(kw)
+        return f(a["x"], a["M"], a["packed"], a["scales"], a["ab"], a["N"], a["K"], a["B"],
+                 a["G"], a["mode"], a["epi"], a["dt"], a["y"], a["s"])
+    assert call(B=5) == 2
+    assert call(dt=2) == 1
+    assert call(epi=3) == 1
+    assert call(y=None) == 1
+    assert call(x=FAKE_ODD) == 2
+    assert call(M=(1 << 24) + 1) == 2
+    assert call(epi=1, N=200) == 2
+    assert call(M=0) == 0
 
 
 def test_oracle_library_builds_and_loads():
