@@ -83,6 +83,7 @@ def _load():
         "cqo_is_monotone": (i32, [u16, u16]),
         "cqo_decode": (None, [P, P, P, i64, i64, i32, i32, i32, P, P, P]),
         "cqo_gemm": (None, [P, i64, P, P, P, i64, i64, i32, i32, i32, P, P, i32]),
+        "cqo_gemm_ex": (None, [P, i64, P, P, P, i64, i64, i32, i32, i32, i32, P, P, i32]),
         "cqo_nearest": (i32, [P, i32, dbl]),
         "cqo_nearest_bruteforce": (i32, [P, i32, dbl]),
         "cqo_fit": (None, [P, i64, i32, i32, i32, P, i32, P, i32, P, i32, i32,
@@ -198,10 +199,14 @@ def decode(packed, scales, ab, N, K, B, G, mode=MIDRISE):
     return w64, w32, w16
 
 
-def gemm(x_bf16bits, packed, scales, ab, N, K, B, G, mode=MIDRISE, nthreads=0):
+def gemm(x_bf16bits, packed, scales, ab, N, K, B, G, mode=MIDRISE, nthreads=0,
+         operand="f64"):
     """y[m][n] = sum_k x[m][k] w[n][k] in FP64 and bound = sum_k |x w|.
 
-    x_bf16bits: uint16 [M][K] (bfloat16 bit patterns)."""
+    x_bf16bits: uint16 [M][K] (bfloat16 bit patterns).
+    operand "f64": w is the exact level; "bf16": w is that level rounded to
+    FP32 and then to BF16, the model-dtype operand of the A16 path
+    ("压缩权重必须“边解码、边计算”")."""
     x = np.ascontiguousarray(x_bf16bits, dtype=np.uint16)
     M = x.shape[0]
     packed = np.ascontiguousarray(packed, dtype=np.uint8)
@@ -209,8 +214,10 @@ def gemm(x_bf16bits, packed, scales, ab, N, K, B, G, mode=MIDRISE, nthreads=0):
     ab = np.ascontiguousarray(ab, dtype=np.uint16)
     y = np.empty((M, N), dtype=np.float64)
     bound = np.empty((M, N), dtype=np.float64)
-    _load().cqo_gemm(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G,
-                     mode, _ptr(y), _ptr(bound), nthreads)
+    if operand not in ("f64", "bf16"):
+        raise ValueError(operand)
+    _load().cqo_gemm_ex(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G,
+                        mode, int(operand == "bf16"), _ptr(y), _ptr(bound), nthreads)
     return y, bound
 
 
@@ -247,8 +254,40 @@ def bf16_bits_to_f64(h: np.ndarray) -> np.ndarray:
 # MoE layer: the composition gate/up -> SwiGLU -> down -> weighted combine
 # --------------------------------------------------------------------------
 
+def f32_down(v: np.ndarray) -> np.ndarray:
+    """Largest FP32 value <= v (elementwise, FP64 in, FP32 out)."""
+    v = np.asarray(v, dtype=np.float64)
+    f = v.astype(np.float32)
+    over = f.astype(np.float64) > v
+    f[over] = np.nextafter(f[over], np.float32(-np.inf))
+    return f
+
+
+def f32_up(v: np.ndarray) -> np.ndarray:
+    """Smallest FP32 value >= v (elementwise, FP64 in, FP32 out)."""
+    v = np.asarray(v, dtype=np.float64)
+    f = v.astype(np.float32)
+    under = f.astype(np.float64) < v
+    f[under] = np.nextafter(f[under], np.float32(np.inf))
+    return f
+
+
+def bf16_rne_of_f32(f: np.ndarray) -> np.ndarray:
+    """FP32 -> BF16 round to nearest even; returns the BF16 values as FP64."""
+    u = np.ascontiguousarray(f, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint32) << 16
+    return r.view(np.float32).astype(np.float64)
+
+
+def bf16_up_bits(v: np.ndarray) -> np.ndarray:
+    """Bit patterns of the smallest BF16 value >= v, for finite v >= 0."""
+    u = f32_up(v).view(np.uint32).astype(np.uint64)
+    r = ((u + 0xFFFF) >> 16).astype(np.uint16)
+    return r
+
+
 def moe_routes(tokens_bf16bits, topk_ids, experts, H, I, G, mode=MIDRISE,
-               routes=None, nthreads=0, rel=2e-3, abs_=1e-6):
+               routes=None, nthreads=0, rel=2e-3, abs_=1e-6, operand="f64"):
     """Per-route outputs of the routed-expert FFN, FP64.
 
     experts[e] = dict(B_gu, packed_gu [2I][H*B/8], scales_gu, ab_gu,
@@ -258,18 +297,29 @@ def moe_routes(tokens_bf16bits, topk_ids, experts, H, I, G, mode=MIDRISE,
     Route r = (t, j) uses expert topk_ids[t][j]:
         gu = W_gu x_t (2I outputs), h = bf16(silu(gu[:I]) * gu[I:]),
         y_r = W_dn h (H outputs).
-    h is rounded to BF16 because the GPU chain stores it in BF16.
+    h is rounded to BF16 because the chain keeps the activation between the
+    two products in the model dtype ("压缩权重必须“边解码、边计算”").
     routes: optional list of flat route indices r = t*k + j to evaluate.
+    operand: the weight operand of both products ("f64" exact levels, or
+    "bf16" the model-dtype operand, see gemm()); rel, abs_: the per-product
+    tolerance that is propagated (2e-3, 1e-6: the contract's GEMM bound for
+    the exact levels; with the BF16 operand, the products differ from the
+    kernel's only by the order of the FP32 sums).
 
     Returns dict r -> (y_r, bound_r, tol_r), all [H] float64:
       bound_r = sum_i |w_dn[n][i] h_i|;
-      tol_r   = the per-GEMM tolerance rel*bound + abs_ of the down product
-                plus the first-order effect of the gate/up product's own
-                tolerance on h: each g, u may be off by e = rel*sum|w x| +
-                abs_, which moves h = silu(g) u by at most
-                |silu'(g)| |u| e_g + |silu(g)| e_u + e_g e_u, and the BF16
-                rounding of a perturbed h may land one BF16 ulp (<= 2^-7 |h|)
-                away; that input difference reaches y_r through |W_dn|."""
+      tol_r   = rel*bound_r + abs_ (the down product's own tolerance) plus
+                (1 + rel) * sum_i |w_dn[n][i]| dh_i, the effect of the
+                gate/up product's tolerance on h.  Each g, u may be off by
+                e = rel*sum|w x| + abs_, which moves the unrounded h =
+                silu(g) u by at most eh = |silu'(g)| |u| e_g + |silu(g)| e_u
+                + e_g e_u (+ FP32 evaluation, 1e-6 |h|).  The GPU's h is the
+                BF16 rounding of a value inside [h - eh, h + eh]; rounding is
+                monotone, so it lies between the roundings of the interval's
+                ends, and dh_i is the larger distance from the oracle's h_i to
+                those two: zero wherever no BF16 rounding boundary falls
+                inside the interval (then both sides round to the same h_i),
+                one BF16 step where one does."""
     T, k = topk_ids.shape
     if routes is None:
         routes = range(T * k)
@@ -284,23 +334,28 @@ def moe_routes(tokens_bf16bits, topk_ids, experts, H, I, G, mode=MIDRISE,
         ex = get(e)
         xs = np.ascontiguousarray(tokens_bf16bits[[r // k for r in rs]])
         gu, bgu = gemm(xs, ex["packed_gu"], ex["scales_gu"], ex["ab_gu"], 2 * I, H,
-                       ex["B_gu"], G, mode, nthreads)
+                       ex["B_gu"], G, mode, nthreads, operand)
         hf = swiglu(gu)
         hb = bf16_round(hf)
         h = bf16_bits_to_f64(hb)
-        y, bnd = gemm(hb, ex["packed_dn"], ex["scales_dn"], ex["ab_dn"], H, I,
-                      ex["B_dn"], G, mode, nthreads)
         g, u = gu[:, :I], gu[:, I:]
         eg, eu = rel * bgu[:, :I] + abs_, rel * bgu[:, I:] + abs_
         sig = 1.0 / (1.0 + np.exp(-g))
         dsilu = np.abs(sig * (1.0 + g * (1.0 - sig)))
         eh = dsilu * np.abs(u) * eg + np.abs(g * sig) * eu + eg * eu + 1e-6 * np.abs(hf)
-        dh = eh + 2.0 ** -7 * (np.abs(h) + eh)
-        wdn, _, _ = decode(ex["packed_dn"], ex["scales_dn"], ex["ab_dn"], H, I, ex["B_dn"], G,
-                           mode)
-        prop = dh @ np.abs(wdn).T
+        lo = bf16_rne_of_f32(f32_down(hf - eh))
+        hi = bf16_rne_of_f32(f32_up(hf + eh))
+        dh = np.maximum(np.maximum(h - lo, hi - h), 0.0)
+        # one pass over W_dn: the rows of h give y and its bound; the rows of
+        # dh (non-negative, rounded up to BF16) give sum_i |w_dn[n][i]| dh_i
+        # from above as their bound
+        xd = np.ascontiguousarray(np.concatenate([hb, bf16_up_bits(dh)]))
+        yy, bb = gemm(xd, ex["packed_dn"], ex["scales_dn"], ex["ab_dn"], H, I,
+                      ex["B_dn"], G, mode, nthreads, operand)
+        n = len(rs)
+        y, bnd, prop = yy[:n], bb[:n], bb[n:]
         for i, r in enumerate(rs):
-            out[r] = (y[i], bnd[i], rel * bnd[i] + abs_ + prop[i])
+            out[r] = (y[i], bnd[i], rel * bnd[i] + abs_ + (1.0 + rel) * prop[i])
     return out
 
 

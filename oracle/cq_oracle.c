@@ -373,6 +373,7 @@ typedef struct {
     const uint16_t *x; int64_t M;
     const uint8_t *packed; const float *scales; const uint16_t *ab;
     int64_t N, K; int B, G, mode;
+    int operand_bf16;
     double *y, *bound;
     int64_t n0, n1;
 } gemm_job;
@@ -386,6 +387,12 @@ static void *gemm_worker(void *p)
         /* this row's exact levels */
         cqo_decode(j->packed + n * rb, j->scales + n * ng, j->ab + n * ng * 2,
                    1, j->K, j->B, j->G, j->mode, wrow, NULL, NULL);
+        /* the model-dtype operand: each level rounded once to FP32, then to
+         * BF16 ([CQ fused]: levels are converted to the model dtype before
+         * the dot product) */
+        if (j->operand_bf16)
+            for (int64_t k = 0; k < j->K; k++)
+                wrow[k] = cqo_bf16_to_double(cqo_float_to_bf16((float)wrow[k]));
         for (int64_t m = 0; m < j->M; m++) {
             double acc = 0.0, bnd = 0.0;
             for (int64_t k = 0; k < j->K; k++) {
@@ -413,19 +420,21 @@ int cqo_num_threads(int requested)
 /*
  * x: bf16 [M][K]; W given packed.  y and bound: double [M][N], where
  * bound[m][n] = sum_k |x[m][k] * w[n][k]| (the scale of the tolerance).
+ * w is the exact FP64 level, or, with operand_bf16, that level rounded to
+ * FP32 and then to BF16 (the operand the tensor cores multiply).
  * Rows of W are split across threads; each output is one plain sequential
  * sum over k.
  */
-void cqo_gemm(const uint16_t *x, int64_t M, const uint8_t *packed, const float *scales,
-              const uint16_t *ab, int64_t N, int64_t K, int B, int G, int mode,
-              double *y, double *bound, int nthreads)
+void cqo_gemm_ex(const uint16_t *x, int64_t M, const uint8_t *packed, const float *scales,
+                 const uint16_t *ab, int64_t N, int64_t K, int B, int G, int mode,
+                 int operand_bf16, double *y, double *bound, int nthreads)
 {
     int T = cqo_num_threads(nthreads);
     if (T > N) T = (int)(N > 0 ? N : 1);
     pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * T);
     gemm_job *jobs = (gemm_job *)malloc(sizeof(gemm_job) * T);
     for (int i = 0; i < T; i++) {
-        gemm_job j = {x, M, packed, scales, ab, N, K, B, G, mode, y, bound,
+        gemm_job j = {x, M, packed, scales, ab, N, K, B, G, mode, operand_bf16, y, bound,
                       N * i / T, N * (i + 1) / T};
         jobs[i] = j;
         pthread_create(&th[i], NULL, gemm_worker, &jobs[i]);
@@ -434,6 +443,14 @@ void cqo_gemm(const uint16_t *x, int64_t M, const uint8_t *packed, const float *
         pthread_join(th[i], NULL);
     free(th);
     free(jobs);
+}
+
+/* The FP64-level product (operand_bf16 = 0). */
+void cqo_gemm(const uint16_t *x, int64_t M, const uint8_t *packed, const float *scales,
+              const uint16_t *ab, int64_t N, int64_t K, int B, int G, int mode,
+              double *y, double *bound, int nthreads)
+{
+    cqo_gemm_ex(x, M, packed, scales, ab, N, K, B, G, mode, 0, y, bound, nthreads);
 }
 
 /* ------------------------------------------------------------------------ */

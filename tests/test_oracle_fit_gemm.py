@@ -49,6 +49,111 @@ def test_gemm_equals_library_matmul_of_decoded(B, G, mode):
     assert np.array_equal(w32, w64.astype(np.float32))
 
 
+@pytest.mark.parametrize("B,G,mode", [(2, 128, 0), (3, 512, 0), (4, 256, 1)])
+def test_gemm_bf16_operand_is_matmul_of_decoded_bf16(B, G, mode):
+    """operand="bf16" multiplies by the decode's BF16 weights (each level
+    rounded to FP32, then to BF16), as a library matmul of cq's decode
+    output does; the FP64-level product differs from it."""
+    N, K, M = 29, 1024, 4
+    codes, packed, s, ab = _rand_matrix(N, K, B, G, mode, seed=40 + B)
+    x = _bf16_act(M, K, seed=41)
+    _, _, w16 = oracle.decode(packed, s, ab, N, K, B, G, mode)
+    wb = oracle.bf16_bits_to_f64(w16)
+    y, bound = oracle.gemm(x, packed, s, ab, N, K, B, G, mode, operand="bf16")
+    xf = oracle.bf16_bits_to_f64(x)
+    assert np.allclose(y, xf @ wb.T, rtol=1e-12, atol=1e-12)
+    assert np.allclose(bound, np.abs(xf) @ np.abs(wb).T, rtol=1e-12, atol=1e-12)
+    y64, _ = oracle.gemm(x, packed, s, ab, N, K, B, G, mode)
+    assert not np.allclose(y, y64, rtol=1e-9, atol=0)
+
+
+def test_directed_rounding_helpers():
+    v = np.concatenate([RNG.normal(size=2000) * 10.0 ** RNG.integers(-30, 30, size=2000),
+                        [0.0, 1.0, -1.0, 1.0 + 2.0 ** -30, 3.0]])
+    lo, hi = oracle.f32_down(v), oracle.f32_up(v)
+    assert np.all(lo.astype(np.float64) <= v) and np.all(hi.astype(np.float64) >= v)
+    # nothing representable in FP32 lies strictly between the result and v
+    assert np.all(np.nextafter(lo, np.float32(np.inf)).astype(np.float64) > v)
+    assert np.all(np.nextafter(hi, np.float32(-np.inf)).astype(np.float64) < v)
+    exact = v.astype(np.float32).astype(np.float64) == v
+    assert np.all(lo[exact] == hi[exact])
+    # RNE FP32 -> BF16 agrees with the oracle's FP64 -> FP32 -> BF16 rounding on FP32 input
+    f = (RNG.normal(size=5000) * 7).astype(np.float32)
+    f = np.concatenate([f, np.float32([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8)])])
+    assert np.array_equal(oracle.bf16_rne_of_f32(f),
+                          oracle.bf16_bits_to_f64(oracle.bf16_round(f.astype(np.float64))))
+    # smallest BF16 value >= v
+    w = np.abs(RNG.normal(size=3000)) * 10.0 ** RNG.integers(-20, 20, size=3000)
+    up = oracle.bf16_bits_to_f64(oracle.bf16_up_bits(w))
+    assert np.all(up >= w)
+    below = oracle.bf16_bits_to_f64(oracle.bf16_up_bits(w) - 1)
+    assert np.all(below < w)
+
+
+def _chain_layer(B=3, H=1024, I=512, E=3, seed=0):
+    exps = []
+    for e in range(E):
+        _, pgu, sgu, agu = _rand_matrix(2 * I, H, B, 128, seed=seed + 10 * e)
+        _, pdn, sdn, adn = _rand_matrix(H, I, B, 128, seed=seed + 10 * e + 5)
+        exps.append(dict(B_gu=B, packed_gu=pgu, scales_gu=sgu, ab_gu=agu,
+                         B_dn=B, packed_dn=pdn, scales_dn=sdn, ab_dn=adn))
+    return exps
+
+
+def _simulated_chain(x, ids, exps, H, I, G, operand, noise, rng, hround="rne", swap=False):
+    """A stand-in for a kernel, on the CPU: the two products with errors of
+    up to `noise` times their tolerance, h evaluated in FP32 and rounded to
+    BF16 (or, to plant a mistake, truncated / with gate and up swapped)."""
+    rel = 2e-3 if operand == "f64" else 2e-5
+    T, k = ids.shape
+    out = {}
+    for r in range(T * k):
+        ex = exps[int(ids[r // k, r % k])]
+        gu, bgu = oracle.gemm(x[r // k:r // k + 1], ex["packed_gu"], ex["scales_gu"],
+                              ex["ab_gu"], 2 * I, H, ex["B_gu"], G, operand=operand)
+        gu = gu + noise * rng.uniform(-1, 1, gu.shape) * (rel * bgu + 1e-6)
+        g, u = gu[0, :I].astype(np.float32), gu[0, I:].astype(np.float32)
+        if swap:
+            g, u = u, g
+        hf = (g / (np.float32(1) + np.exp(-g)) * u).astype(np.float32)
+        if hround == "rne":
+            hb = oracle.bf16_round(hf.astype(np.float64))
+        else:   # truncation toward zero
+            hb = (hf.view(np.uint32) >> 16).astype(np.uint16)
+        y, by = oracle.gemm(hb[None, :], ex["packed_dn"], ex["scales_dn"], ex["ab_dn"], H, I,
+                            ex["B_dn"], G, operand=operand)
+        out[r] = y[0] + noise * rng.uniform(-1, 1, H) * (rel * by[0] + 1e-6)
+    return out
+
+
+@pytest.mark.parametrize("operand", ["f64", "bf16"])
+def test_moe_chain_tolerance_accepts_a_correct_chain_and_rejects_planted_mistakes(operand):
+    """The chain tolerance of moe_routes: a CPU stand-in for a kernel whose
+    products err by up to half their own tolerance (in either direction)
+    and which rounds h to BF16 correctly passes; the same chain with h
+    truncated instead of rounded (BF16-operand check), or with gate and up
+    swapped, fails."""
+    H, I, G, T, k, E = 1024, 512, 128, 3, 2, 3
+    exps = _chain_layer(3, H, I, E, seed=300)
+    x = _bf16_act(T, H, seed=301)
+    ids, _ = synthetic.routing_uniform(302, T, E, k)
+    ids = ids.numpy()
+    rel, abs_ = (2e-3, 1e-6) if operand == "f64" else (2e-5, 1e-7)
+    ref = oracle.moe_routes(x, ids, exps, H, I, G, rel=rel, abs_=abs_, operand=operand)
+    rng = np.random.default_rng(303)
+
+    def worst(sim):
+        return max(float(np.max(np.abs(sim[r] - ref[r][0]) / ref[r][2])) for r in ref)
+
+    assert worst(_simulated_chain(x, ids, exps, H, I, G, operand, 0.5, rng)) <= 1.0
+    assert worst(_simulated_chain(x, ids, exps, H, I, G, operand, 0.0, rng, swap=True)) > 1.0
+    if operand == "bf16":
+        assert worst(_simulated_chain(x, ids, exps, H, I, G, operand, 0.0, rng,
+                                      hround="trunc")) > 1.0
+        # far tighter than the contract's bound on a typical element
+        assert np.median(ref[0][2] / ref[0][1]) < 2e-3
+
+
 @pytest.mark.parametrize("B", [2, 3, 4])
 def test_gemm_uniform_case_is_integer_dequant_matmul(B):
     """With every group at a = 1, b = 0 the GEMM is the textbook symmetric
