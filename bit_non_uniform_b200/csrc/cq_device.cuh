@@ -34,6 +34,12 @@ enum WaitSite : int {
   SITE_GV_TABLE_FULL = 13,
   SITE_GV_SLOT = 14,
   SITE_GV_X = 15,
+  // narrow-row kernel
+  SITE_NR_XEMPTY = 16,
+  SITE_NR_CEMPTY = 17,
+  SITE_NR_CFULL = 18,
+  SITE_NR_XFULL = 19,
+  SITE_NR_PARTIAL = 45,   // the owner of a shared row block waiting for the other parts
 };
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -167,6 +173,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
       "[%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+// 3-D tiled tensor copy global -> shared (no multicast).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int32_t c0,
+                                            int32_t c1, int32_t c2, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
       : "memory");
 }
 

@@ -6,6 +6,7 @@
 #include "cq_hooks.h"
 #include "cq_engine.cuh"
 #include "cq_gemv_launch.cuh"
+#include "cq_narrow_launch.cuh"
 #include "cq_host.h"
 
 namespace cq {
@@ -54,10 +55,23 @@ static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int B, int epilogue, 
   return g;
 }
 
+// Which kernel runs a cq_gemm call: the narrow-row kernel for up to 16 tokens
+// when its plan fits, else the decode-sized GEMV (up to 2 tokens), else the
+// tensor-core engine.  (The test hook may force one of them.)
+enum GemmPath { PATH_AUTO = 0, PATH_NARROW = 1, PATH_GEMV = 2, PATH_ENGINE = 3 };
+
 // Scratch bytes of whichever path gemm_impl takes for this problem.
 static void gemm_scratch(int64_t M, int64_t N, int64_t K, int B, int G, int epilogue, int sms,
-                         size_t* counter_bytes, size_t* total) {
-  const GvPlan v = plan_gemv(M, N, K, B, G, epilogue, sms);
+                         size_t* counter_bytes, size_t* total, int path = PATH_AUTO) {
+  if (path == PATH_AUTO || path == PATH_NARROW) {
+    const NrPlan nv = plan_narrow(M, N, K, B, G, epilogue, sms);
+    if (nv.use) {
+      *counter_bytes = nv.ws_counter_bytes;
+      *total = nv.ws_counter_bytes + nv.ws_partial_bytes;
+      return;
+    }
+  }
+  const GvPlan v = path == PATH_ENGINE ? GvPlan{} : plan_gemv(M, N, K, B, G, epilogue, sms);
   if (v.use) {
     *counter_bytes = v.ws_counter_bytes;
     *total = v.ws_counter_bytes + v.ws_partial_bytes;
@@ -129,14 +143,27 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
               const uint16_t* ab, int64_t N, int64_t K, int B, int G, int grid_mode,
               int epilogue, int out_dtype, void* y, void* workspace, size_t ws_bytes,
               cudaStream_t stream, uint64_t timeout_ns, int debug_skip,
-              uint64_t* trace = nullptr) {
+              uint64_t* trace = nullptr, int path = PATH_AUTO) {
   int st = validate_gemm(x, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype,
                          y);
   if (st != CQ_OK) return st;
   if (M == 0 || N == 0) return CQ_OK;
   const int sms = num_sms();
   if (sms <= 0) return CQ_ERR_CUDA;
-  const GvPlan v = debug_skip ? GvPlan{} : plan_gemv(M, N, K, B, G, epilogue, sms);
+  if (debug_skip) path = PATH_ENGINE;
+  if (path == PATH_AUTO || path == PATH_NARROW) {
+    const NrPlan nv = plan_narrow(M, N, K, B, G, epilogue, sms);
+    if (nv.use) {
+      const size_t need = nv.ws_counter_bytes + nv.ws_partial_bytes;
+      if (ws_bytes < need || !workspace) return CQ_ERR_WORKSPACE;
+      if (!aligned(workspace, 16)) return CQ_ERR_UNSUPPORTED;
+      return run_narrow(nv, x, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue,
+                        out_dtype, y, workspace, stream, timeout_ns, trace);
+    }
+    if (path == PATH_NARROW) return CQ_ERR_UNSUPPORTED;
+  }
+  const GvPlan v = path == PATH_ENGINE ? GvPlan{} : plan_gemv(M, N, K, B, G, epilogue, sms);
+  if (path == PATH_GEMV && !v.use) return CQ_ERR_UNSUPPORTED;
   if (v.use)
     return run_gemv(v, x, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype, y,
                     stream, timeout_ns, trace);
@@ -190,13 +217,13 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
 }
 
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K, int B, int G, int epilogue,
-                           int sms) {
+                           int sms, int path = PATH_AUTO) {
   if (M <= 0 || N <= 0 || K <= 0 || K % kSlice != 0 || G <= 0 || G % kSlice != 0 ||
       K % G != 0 || M > (int64_t)1 << 24 || N > (int64_t)1 << 30 ||
       ((M + 15) / 16) * ((N + kRows - 1) / kRows) >= ((int64_t)1 << 31))
     return 0;                                     // cq_gemm rejects these shapes
   size_t counters = 0, total = 0;
-  gemm_scratch(M, N, K, B, G, epilogue, sms, &counters, &total);
+  gemm_scratch(M, N, K, B, G, epilogue, sms, &counters, &total, path);
   return total;
 }
 
@@ -241,4 +268,24 @@ extern "C" CQ_API int cq_test_gemm_bounded(const uint16_t* x, int64_t M, const u
   return gemm_impl(x, M, packed, scales, ab, N, K, B, G, CQ_GRID_MIDRISE, CQ_EPI_NONE,
                    CQ_DTYPE_F32, y, workspace, ws_bytes, static_cast<cudaStream_t>(stream),
                    timeout_ns, skip_first_stage);
+}
+
+// Test hook (declared in cq_hooks.h): cq_gemm on a chosen kernel, and the
+// workspace that choice needs.
+extern "C" CQ_API size_t cq_test_gemm_path_workspace_size(int64_t M, int64_t N, int64_t K, int B,
+                                                         int G, int epilogue, int path) {
+  int sms = num_sms();
+  if (sms <= 0) sms = 148;
+  return gemm_workspace_size(M, N, K, B, G, epilogue, sms, path);
+}
+
+extern "C" CQ_API int cq_test_gemm_path(const uint16_t* x, int64_t M, const uint8_t* packed,
+                                        const float* scales, const uint16_t* ab, int64_t N,
+                                        int64_t K, int B, int G, int grid_mode, int epilogue,
+                                        int out_dtype, void* y, void* workspace, size_t ws_bytes,
+                                        int path, void* stream) {
+  if (path < PATH_AUTO || path > PATH_ENGINE) return CQ_ERR_INVALID_ARG;
+  return gemm_impl(x, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype, y,
+                   workspace, ws_bytes, static_cast<cudaStream_t>(stream), kDefaultTimeoutNs, 0,
+                   nullptr, path);
 }

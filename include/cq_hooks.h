@@ -42,6 +42,21 @@ CQ_API int cq_test_gemm_bounded(const uint16_t *x, int64_t M, const uint8_t *pac
                                 int B, int G, void *y, void *workspace, size_t ws_bytes,
                                 uint64_t timeout_ns, int skip_first_stage, void *stream);
 
+/*
+ * cq_test_gemm_path -- cq_gemm on a chosen kernel: path 0 = the one cq_gemm
+ * picks, 1 = the narrow-row kernel (M <= 16), 2 = the decode-sized GEMV
+ * (M <= 2), 3 = the tensor-core engine.  A path that does not take the
+ * problem returns CQ_ERR_UNSUPPORTED.  cq_test_gemm_path_workspace_size gives
+ * the workspace that path needs.  Used to check the kernels against each
+ * other on the same inputs.
+ */
+CQ_API size_t cq_test_gemm_path_workspace_size(int64_t M, int64_t N, int64_t K, int B, int G,
+                                               int epilogue, int path);
+CQ_API int cq_test_gemm_path(const uint16_t *x, int64_t M, const uint8_t *packed,
+                             const float *scales, const uint16_t *ab, int64_t N, int64_t K,
+                             int B, int G, int grid_mode, int epilogue, int out_dtype, void *y,
+                             void *workspace, size_t ws_bytes, int path, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

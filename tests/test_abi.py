@@ -40,7 +40,8 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_hooks_are_declared_and_exported(lib):
     hooks = _declared_symbols("cq_hooks.h")
-    assert hooks == ["cq_test_gemm_bounded", "cq_trace_gemm"]
+    assert hooks == ["cq_test_gemm_bounded", "cq_test_gemm_path",
+                     "cq_test_gemm_path_workspace_size", "cq_trace_gemm"]
     for s in hooks:
         assert hasattr(lib, s), s
 

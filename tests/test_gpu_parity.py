@@ -217,6 +217,52 @@ def test_gemv_matches_decoded_bf16_matmul(cq, M, B, epi):
         assert torch.allclose(h, href, rtol=1e-4, atol=1e-5)
 
 
+PATH_CASES = [
+    # M,  N,    K,    B, G,   mode, epi
+    (1,  7168, 3072, 3, 512, 0, 0),
+    (2,  1000, 2048, 4, 256, 1, 0),
+    (8,  512,  1536, 2, 128, 0, 1),
+    (16, 384,  1024, 3, 512, 0, 0),
+    (11, 257,  512,  2, 512, 0, 0),
+]
+
+
+@pytest.mark.parametrize("M,N,K,B,G,mode,epi", PATH_CASES)
+def test_kernels_agree_on_the_decoded_bf16_operand(cq, M, N, K, B, G, mode, epi):
+    """Every kernel that takes a problem (narrow-row for M <= 16, the GEMV for
+    M <= 2, the tensor-core engine for any M) equals the matmul of cq_decode's
+    BF16 weights up to FP32 summation order, and the narrow kernel is run to
+    run deterministic."""
+    codes, s, ab = make_matrix(("paths", M, N, B), N, K, B, G, mode)
+    pk, sd, abd = to_dev(codes, s, ab, B, cq)
+    x = synthetic.activations(31 + M, M, K).cuda()
+    w = cq.cq_decode(pk, sd, abd, K, B, G, mode, cq.BF16).double()
+    ref = x.double() @ w.T
+    bound = x.double().abs() @ w.abs().T
+    if epi:
+        g, u = ref[:, : N // 2], ref[:, N // 2:]
+        ref = g / (1 + torch.exp(-g)) * u
+    ran = 0
+    for path in (cq.PATH_NARROW, cq.PATH_GEMV, cq.PATH_ENGINE):
+        try:
+            y = cq.gemm_on_path(path, x, pk, sd, abd, N, K, B, G, mode, epi).double()
+        except cq.CQError as e:
+            assert e.status == 2 and (path != cq.PATH_ENGINE)
+            continue
+        ran += 1
+        if epi:
+            assert torch.allclose(y, ref, rtol=1e-4, atol=1e-5), f"path {path}"
+        else:
+            err = (y - ref).abs()
+            assert torch.all(err <= 1e-5 * bound + 1e-7), f"path {path}: {float(err.max())}"
+        if path == cq.PATH_NARROW:
+            y2 = cq.gemm_on_path(path, x, pk, sd, abd, N, K, B, G, mode, epi).double()
+            assert torch.equal(y, y2)
+    assert ran >= 2
+    torch.cuda.synchronize()
+    assert cq.device_error() == (0, 0)
+
+
 def check_swiglu(y_gpu, yr, bd, dt):
     n2 = yr.shape[1] // 2
     g, u = yr[:, :n2], yr[:, n2:]
