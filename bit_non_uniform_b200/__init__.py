@@ -78,6 +78,12 @@ def lib():
         "cq_get_device_error": (i32, [P, ctypes.POINTER(ctypes.c_int)]),
         "cq_test_gemm_bounded": (i32, [P, i64, P, P, P, i64, i64, i32, i32, P, P, sz, u64,
                                        i32, P]),
+        "cq_test_gemm_path_workspace_size": (sz, [i64, i64, i64, i32, i32, i32, i32]),
+        "cq_quant_rows": (i32, [P, i64, i64, P, P, P]),
+        "cq_gemm_a8_workspace_size": (sz, [i64, i64, i64, i32, i32, i32]),
+        "cq_gemm_a8": (i32, [P, i64, P, P, P, i64, i64, i32, i32, i32, i32, i32, P, P, sz, P]),
+        "cq_test_gemm_path": (i32, [P, i64, P, P, P, i64, i64, i32, i32, i32, i32, i32, P, P,
+                                    sz, i32, P]),
     }
     for name, (res, args) in sigs.items():
         f = getattr(L, name)
@@ -164,6 +170,28 @@ def cq_gemm(x, packed, scales, ab, N: int, K: int, B: int, G: int, mode: int = M
     return out
 
 
+# kernels of cq_gemm (test hook cq_test_gemm_path)
+PATH_AUTO, PATH_NARROW, PATH_GEMV, PATH_ENGINE = 0, 1, 2, 3
+
+
+def gemm_on_path(path: int, x, packed, scales, ab, N: int, K: int, B: int, G: int,
+                 mode: int = MIDRISE, epilogue: int = EPI_NONE, out_dtype: int = F32,
+                 stream=None):
+    """cq_gemm on a chosen kernel (a test hook); raises CQError with status 2
+    when that kernel does not take the problem."""
+    _need_cuda(x, packed, scales, ab)
+    M = x.shape[0]
+    ncol = N // 2 if epilogue == EPI_SWIGLU else N
+    dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+    out = torch.empty((M, ncol), dtype=dt, device=x.device)
+    n = int(lib().cq_test_gemm_path_workspace_size(M, N, K, B, G, epilogue, path))
+    ws = torch.zeros(max(n, 16), dtype=torch.uint8, device=x.device)
+    _check(lib().cq_test_gemm_path(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G,
+                                   mode, epilogue, out_dtype, _ptr(out), _ptr(ws), ws.numel(),
+                                   path, _stream(stream)), "cq_test_gemm_path")
+    return out
+
+
 def cq_gemm_noalloc(x, packed, scales, ab, N: int, K: int, B: int, G: int,
                     mode: int = MIDRISE, epilogue: int = EPI_NONE, out_dtype: int = F32,
                     out=None, stream=None):
@@ -177,6 +205,42 @@ def cq_gemm_noalloc(x, packed, scales, ab, N: int, K: int, B: int, G: int,
     _check(lib().cq_gemm_noalloc(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G,
                                  mode, epilogue, out_dtype, _ptr(out), _stream(stream)),
            "cq_gemm_noalloc")
+    return out
+
+
+def gemm_a8_workspace_size(M, N, K, B, G, epilogue=EPI_NONE) -> int:
+    return int(lib().cq_gemm_a8_workspace_size(M, N, K, B, G, epilogue))
+
+
+def cq_quant_rows(x, stream=None):
+    """Per-row dynamic INT8 quantization: (xq int8 [M][K], absmax f32 [M])."""
+    _need_cuda(x)
+    assert x.dtype == torch.bfloat16 and x.is_contiguous()
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    absmax = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib().cq_quant_rows(_ptr(x), M, K, _ptr(xq), _ptr(absmax), _stream(stream)),
+           "cq_quant_rows")
+    return xq, absmax
+
+
+def cq_gemm_a8(x, packed, scales, ab, N: int, K: int, B: int, G: int, mode: int = MIDRISE,
+               epilogue: int = EPI_NONE, out_dtype: int = F32, out=None, workspace=None,
+               stream=None):
+    """Dynamic-A8 y = x W^T: x quantized per row to INT8 inside the call."""
+    _need_cuda(x, packed, scales, ab)
+    assert x.dtype == torch.bfloat16 and x.is_contiguous()
+    M = x.shape[0]
+    ncol = N // 2 if epilogue == EPI_SWIGLU else N
+    if out is None:
+        dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+        out = torch.empty((M, ncol), dtype=dt, device=x.device)
+    if workspace is None:
+        n = gemm_a8_workspace_size(M, N, K, B, G, epilogue)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=x.device)
+    _check(lib().cq_gemm_a8(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G, mode,
+                            epilogue, out_dtype, _ptr(out), _ptr(workspace),
+                            workspace.numel(), _stream(stream)), "cq_gemm_a8")
     return out
 
 

@@ -14,7 +14,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libcq.so")
 SOURCES = ["cq_lib.cu"]
-HEADERS = ["cq_gemv.cuh", "cq_gemv_launch.cuh", "cq_api.cu", "cq_gemm.cu", "cq_moe.cu", "cq_noalloc.cu", "cq_device.cuh", "cq_engine.cuh",
+HEADERS = ["cq_gemv.cuh", "cq_gemv_launch.cuh", "cq_narrow.cuh", "cq_narrow_launch.cuh", "cq_api.cu", "cq_gemm.cu", "cq_moe.cu", "cq_noalloc.cu", "cq_a8.cu", "cq_a8.cuh", "cq_device.cuh", "cq_engine.cuh",
            "cq_host.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

@@ -4,3 +4,4 @@
 #include "cq_gemm.cu"
 #include "cq_moe.cu"
 #include "cq_noalloc.cu"
+#include "cq_a8.cu"

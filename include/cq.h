@@ -119,13 +119,17 @@ CQ_API int cq_decode(const uint8_t *packed, const float *scales, const uint16_t 
  *              counters that must be zero before the first call that uses
  *              the buffer; every completed call leaves them zero again.
  * Calls that share one workspace must not overlap on the GPU.
- * Paths: M <= 2 runs the decode-sized GEMV kernel (no workspace: size 0);
- * M >= 3 runs the tensor-core engine (128-row weight tiles, 16- to
- * 192-token activation tiles, stream-K over the K slices, partial tiles
- * summed in a fixed order).  Results are run-to-run deterministic.  Both
- * kernels are launched with programmatic dependent launch: their setup may
- * overlap the end of the preceding kernel in the stream, and they read no
- * caller memory before that kernel has completed (stream order holds).
+ * Paths: M <= 16 with K a multiple of 512 runs the narrow-row kernel
+ * ([CQ] "压缩权重必须“边解码、边计算”": the narrow-row GEMV; register-operand
+ * tensor-core MMAs, 16-row x one-slice work units split evenly over the SMs,
+ * row blocks shared by two CTAs summed through the workspace); other M <= 2
+ * shapes run the decode-sized GEMV kernel (no workspace); everything else
+ * runs the tensor-core engine (128-row weight tiles, 16- to 192-token
+ * activation tiles, stream-K over the K slices, partial tiles summed in a
+ * fixed order).  Results are run-to-run deterministic.  All three kernels
+ * are launched with programmatic dependent launch: their setup may overlap
+ * the end of the preceding kernel in the stream, and they read no caller
+ * memory before that kernel has completed (stream order holds).
  */
 CQ_API size_t cq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int B, int G,
                               int epilogue);
@@ -144,7 +148,8 @@ CQ_API int cq_gemm(const uint16_t *x, int64_t M, const uint8_t *packed, const fl
  * a calling convenience).
  *   Scratch: a fixed 4 MiB array inside libcq (every GPU that loads the
  *   library holds it until the process exits), enough for any M <= 16 on a
- *   148-SM B200; a problem that needs more returns CQ_ERR_WORKSPACE.
+ *   148-SM B200 (narrow-row kernel or engine); a problem that needs more
+ *   returns CQ_ERR_WORKSPACE.
  *   The first call on a device looks up that array's device address (a CUDA
  *   runtime query, which also loads libcq's device code there) and caches
  *   it with the device's context; make that first call before any stream
@@ -160,6 +165,43 @@ CQ_API int cq_gemm_noalloc(const uint16_t *x, int64_t M, const uint8_t *packed,
                            const float *scales, const uint16_t *ab, int64_t N, int64_t K, int B,
                            int G, int grid_mode, int epilogue, int out_dtype, void *y,
                            void *stream);
+
+/*
+ * Dynamic A8 ([CQ] "一份 checkpoint，同时服务 A16 与 Dynamic A8"): the same
+ * checkpoint served with INT8 activations.  The article's carrier and
+ * activation formulas were lost in extraction; this library reads them as
+ *   carrier(u) = RNE(127 * sign(k) * q(t)) (q in FP64), saturated to +-127,
+ *   xq[m][k]   = RNE(x[m][k] * RN_fp32(127 / absmax[m])), saturated to
+ *                +-127, absmax[m] = max_k |x[m][k]| (a zero row gives zeros),
+ *   y[m][n]    = sum_g (absmax[m] / 127) * (s[n][g] / 127) * acc[m][n][g],
+ *                acc the exact integer dot product of group g.
+ *
+ * cq_quant_rows -- per-row INT8 quantization of bfloat16 activations.
+ *   x      bfloat16 [M][K];  xq int8 [M][K] (output);  absmax float [M] (output)
+ * Bit-exact: the decisions are taken in FP32 as written above.
+ */
+CQ_API int cq_quant_rows(const uint16_t *x, int64_t M, int64_t K, int8_t *xq, float *absmax,
+                         void *stream);
+
+/*
+ * cq_gemm_a8 -- the Dynamic-A8 GEMM: x is quantized per row inside the call
+ * (into the workspace), the codes are decoded to their INT8 carriers tile by
+ * tile on chip, the integer dot products run on the tensor cores
+ * (tcgen05.mma kind::i8, INT32 accumulators in tensor memory) and are
+ * scaled once per group in FP32 ([CQ] "实验结果 2. H200 内核交叉点": the A8
+ * path wins from M = 64 on).  Arguments, layouts, epilogues and output
+ * dtypes as cq_gemm; the workspace (cq_gemm_a8_workspace_size bytes, 256-byte
+ * aligned) holds the quantized activations, their row maxima and the
+ * stream-K scratch; its counters are cleared by each call.  Calls that share
+ * one workspace must not overlap on the GPU.  B in {2,3,4}; run-to-run
+ * deterministic.
+ */
+CQ_API size_t cq_gemm_a8_workspace_size(int64_t M, int64_t N, int64_t K, int B, int G,
+                                        int epilogue);
+CQ_API int cq_gemm_a8(const uint16_t *x, int64_t M, const uint8_t *packed, const float *scales,
+                      const uint16_t *ab, int64_t N, int64_t K, int B, int G, int grid_mode,
+                      int epilogue, int out_dtype, void *y, void *workspace, size_t ws_bytes,
+                      void *stream);
 
 /*
  * One quantized matrix of an expert (HOST-side description, device pointers).
