@@ -151,6 +151,23 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 
+// 32-bit global load through the read-only path whose place in the
+// instruction stream is kept (volatile): issued before the loads after it.
+__device__ __forceinline__ uint32_t ldg_u32_ordered(const void* ptr) {
+  uint32_t v;
+  asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(ptr));
+  return v;
+}
+
+// 16-byte global load of data read once (not kept in L1).
+__device__ __forceinline__ uint4 ldg_stream16(const void* ptr) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(ptr));
+  return v;
+}
+
 // 16-byte asynchronous copy global -> shared through L2 only (cp.async.cg).
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");

@@ -38,12 +38,15 @@
 // does it last) adds them in CTA order.  Results are run-to-run
 // deterministic.
 //
-// Roles: eight compute warps (tables, decode + MMA, sums, epilogue) and one
-// producer warp whose first lane keeps two TMA rings full: code stages (one
-// unit each, a 3-D/4-D box of 16 rows x 4 quarters x one slice) and
-// activation stages (one slice step of every token, a 4-D box that lands
-// interleaved as [k pair][token][quarter][8 values], so a warp's 16-byte
-// activation loads are conflict free).
+// Loads.  Each warp loads the codes of its own units straight into registers
+// with 16-byte global loads (the lane's two rows of one slice of its
+// quarter), ahead of its decoding, and the CTA stages its activations once,
+// with 16-byte asynchronous copies, as [slice step][k pair][token][quarter]
+// [8 values], so that a warp's 16-byte activation loads are conflict free.
+// (Box copies of 16 rows x 4 quarters x one 48-byte slice came in too
+// slowly: the copy engine handles such short rows at a few bytes per
+// cycle.)  No shared-memory ring, no producer warp: eight warps build the
+// tables, decode, multiply and finish row blocks.
 //
 // This is the narrow-row GEMV of the article's A16 path ("压缩权重必须“边解码、
 // 边计算”"): codes and group parameters -> levels generated in the tile ->
@@ -58,21 +61,16 @@
 
 namespace cq {
 
-constexpr int kNrCompute = 8;                   // compute warps
-constexpr int kNrProducerWarp = 8;
-constexpr int kNrThreads = (kNrCompute + 1) * 32;
+constexpr int kNrCompute = 8;                   // warps
+constexpr int kNrThreads = kNrCompute * 32;
 constexpr int kNrMaxRbl = 8;                    // row blocks one CTA may touch
 constexpr int kNrMaxUnits = 96;                 // units one CTA may own
 constexpr int kNrMaxJ = 64;                     // slice steps per quarter (K <= 32768)
-constexpr int kNrMaxCS = 96;                    // code stages
-constexpr int kNrMaxXS = 64;                    // activation stages
-// barriers, flags, the issue tags of the two rings, and per row block the
-// units of the CTA and how many of them are done
-constexpr int kNrBarBytes =
-    8 * (2 * kNrMaxCS + 2 * kNrMaxXS) + 64 + 4 * (kNrMaxCS + kNrMaxXS) + 8 * kNrMaxRbl;
-// the processing order of a CTA's units, its inverse (unit of (rbl, j)) and
-// the slice step of each activation stage
-constexpr int kNrOrderBytes = 4 * (kNrMaxUnits + kNrMaxRbl * kNrMaxJ + kNrMaxXS);
+constexpr int kNrPreItems = 4;                  // table items per thread loaded up front
+// flags, and per row block the units of the CTA and how many of them are done
+constexpr int kNrBarBytes = 64 + 8 * kNrMaxRbl;
+// the processing order of a CTA's units and its inverse (unit of (rbl, j))
+constexpr int kNrOrderBytes = 4 * (kNrMaxUnits + kNrMaxRbl * kNrMaxJ);
 
 struct NarrowParams {
   int N, K, G, mode, epilogue, out_bf16;
@@ -86,12 +84,13 @@ struct NarrowParams {
   int P;               // CTAs
   int max_rbl;         // row blocks of the largest CTA share (table layout)
   int max_units;       // units of the largest CTA share (slot layout)
-  int CS, XS;          // code / activation stages
-  int resident_x;      // 1: every slice step's activations stay loaded (XS = Q)
-  int tbl_off, code_off, x_off, slot_off;   // shared-memory layout (bytes from the base)
+  int tbl_off, x_off, slot_off;   // shared-memory layout (bytes from the base)
   int smem_bytes;
+  const uint8_t* packed;          // [N][K*B/8]
+  int64_t row_bytes;              // K*B/8
   const float* scales;
   const uint32_t* ab;  // (a | b << 16), fp16 bits
+  const uint16_t* x;   // [M][K] bf16
   void* y;
   int64_t ldy;
   int* counter;        // [n_rb] row blocks shared by CTAs (zero between calls)
@@ -105,31 +104,7 @@ template <int B>
 struct NrCfg {
   static constexpr int E = (B == 3) ? 64 : 16;     // table entries per (row, group)
   static constexpr int SLICE = 16 * B;             // bytes of one row's slice
-  static constexpr int STAGE = 16 * 4 * SLICE;     // one unit's codes
 };
-
-// Wait (bounded) until a ring stage's issue tag shows `use`: the producer
-// writes the tag when it issues that use into the stage, after the stage's
-// previous use has landed and been released.  A consumer then waits on the
-// stage's full barrier with the parity of `use` knowing that the barrier's
-// pending phase is exactly that use (a parity wait alone cannot tell phases
-// two apart, and a consumer may reach its unit before the stage's previous
-// use has even landed).
-__device__ __forceinline__ bool nr_wait_tag(const volatile int* tag, int use, volatile int* abort,
-                                            uint64_t timeout_ns, int site) {
-  if (*tag == use) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    __nanosleep(64);
-    if (*tag == use) return true;
-    if (*abort) return false;
-    if (globaltimer() - t0 > timeout_ns) {
-      *abort = site;
-      atomicCAS(&g_device_error, 0, site);
-      return false;
-    }
-  }
-}
 
 #define NR_STAMP(k)                                                                 \
   do {                                                                              \
@@ -142,6 +117,23 @@ __device__ __forceinline__ int nr_begin(int U, int P, int c) {
 }
 __device__ __forceinline__ int nr_owner(int U, int P, int u) {
   return static_cast<int>((static_cast<int64_t>(u + 1) * P - 1) / U);
+}
+
+// Table item id of a CTA (block = id / 32, lane = id % 32): the weight row and
+// group its table holds; false when there is none (rows past N, groups past
+// the lane column's quarter), whose table is zero.
+__device__ __forceinline__ bool nr_item(const NarrowParams& p, int rb_lo, int id, int& row,
+                                        int& grp) {
+  const int ln = id & 31;
+  const int blk = id >> 5;
+  const int lgi = blk % p.L;
+  const int it = (blk / p.L) & 1;
+  const int rb = rb_lo + blk / (2 * p.L);
+  const int g = ln >> 2, c = ln & 3;
+  row = gv_row(p.N, p.epilogue, rb, it, g);
+  grp = (c * p.Q) / p.spc + lgi;
+  const int grp_last = ((c + 1) * p.Q - 1) / p.spc;
+  return row < p.N && grp <= grp_last && grp < p.ng && rb < p.n_rb;
 }
 
 // First group of quarter c and the table block (0..L-1) of slice step j in it.
@@ -227,8 +219,10 @@ __device__ __noinline__ bool nr_finish_row_block(const NarrowParams& p, int cta,
     __threadfence();
     __syncwarp();
     if (lane == 0) atomicAdd(p.counter + rb, 1);
+    if (lane == 0 && p.trace) p.trace[blockIdx.x * 64 + 40] = clock64();
     return true;
   }
+  if (lane == 0 && p.trace) p.trace[blockIdx.x * 64 + 41] = clock64();
   // the owner: the other CTAs did their part of rb first
   bool ok = true;
   if (lane == 0) {
@@ -249,6 +243,7 @@ __device__ __noinline__ bool nr_finish_row_block(const NarrowParams& p, int cta,
     }
   }
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (lane == 0 && p.trace) p.trace[blockIdx.x * 64 + 42] = clock64();
   if (!ok) return false;
   __threadfence();
   for (int cc = c_lo + 1; cc <= c_hi; ++cc) {
@@ -262,46 +257,62 @@ __device__ __noinline__ bool nr_finish_row_block(const NarrowParams& p, int cta,
   return true;
 }
 
+// The lane's codes of one unit: rows g (c0) and g+8 (c1) of the row block,
+// slice j of quarter c, B 16-byte vectors each, straight from global memory
+// (not kept in L1: every byte is read once).  Rows past N read as zero.
+template <int B>
+__device__ __forceinline__ void nr_load_codes(const NarrowParams& p, int rb, int j, int g, int c,
+                                              uint32_t (&c0)[4 * B], uint32_t (&c1)[4 * B]) {
+  const int r0 = gv_row(p.N, p.epilogue, rb, 0, g);
+  const int r1 = gv_row(p.N, p.epilogue, rb, 1, g);
+  const int64_t off = static_cast<int64_t>(c) * (p.row_bytes / 4) + j * (16 * B);
+#pragma unroll
+  for (int v = 0; v < B; ++v) {
+    uint4 q0 = make_uint4(0u, 0u, 0u, 0u), q1 = make_uint4(0u, 0u, 0u, 0u);
+    if (r0 < p.N)
+      q0 = ldg_stream16(p.packed + static_cast<int64_t>(r0) * p.row_bytes + off + 16 * v);
+    if (r1 < p.N)
+      q1 = ldg_stream16(p.packed + static_cast<int64_t>(r1) * p.row_bytes + off + 16 * v);
+    c0[4 * v + 0] = q0.x;
+    c0[4 * v + 1] = q0.y;
+    c0[4 * v + 2] = q0.z;
+    c0[4 * v + 3] = q0.w;
+    c1[4 * v + 0] = q1.x;
+    c1[4 * v + 1] = q1.y;
+    c1[4 * v + 2] = q1.z;
+    c1[4 * v + 3] = q1.w;
+  }
+}
+
 template <int B, int MT>
 __global__ void __launch_bounds__(kNrThreads, 1)
-    narrow_kernel(const __grid_constant__ NarrowParams p,
-                  const __grid_constant__ CUtensorMap wmap,
-                  const __grid_constant__ CUtensorMap xmap) {
+    narrow_kernel(const __grid_constant__ NarrowParams p) {
   using C = NrCfg<B>;
   constexpr int E = C::E;
   constexpr int NV = 4 * (MT / 8);                  // partial floats per lane and unit
+  constexpr int NB = B == 4 ? 1 : 2;                // units of codes loaded ahead
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   // the tables are addressed by OR: their base is aligned to a table block
   const uint32_t base = (raw + (E * 128u - 1u)) & ~(E * 128u - 1u);
   uint8_t* const gbase = smem_raw + (base - raw);
   const uint32_t tbl0 = base + p.tbl_off;
-  const uint32_t codes0 = base + p.code_off;
   const uint32_t xs0 = base + p.x_off;
-  const uint32_t bars = raw + static_cast<uint32_t>(p.smem_bytes - kNrBarBytes - kNrOrderBytes);
-  const uint32_t bar_cfull = bars;                           // [CS]
-  const uint32_t bar_cempty = bar_cfull + 8 * kNrMaxCS;      // [CS]
-  const uint32_t bar_xfull = bar_cempty + 8 * kNrMaxCS;      // [XS]
-  const uint32_t bar_xempty = bar_xfull + 8 * kNrMaxXS;      // [XS]
-  volatile int* const flags =
-      reinterpret_cast<volatile int*>(smem_raw + (bar_xempty + 8 * kNrMaxXS - raw));
-  volatile int* const ctag = flags + 16;                    // [CS] unit issued into a code stage
-  volatile int* const xtag = ctag + kNrMaxCS;               // [XS] use issued into an x stage
-  int* const cnt_rb = const_cast<int*>(xtag + kNrMaxXS);    // [rbl] the CTA's units of it
+  const uint32_t fl = raw + static_cast<uint32_t>(p.smem_bytes - kNrBarBytes - kNrOrderBytes);
+  volatile int* const flags = reinterpret_cast<volatile int*>(smem_raw + (fl - raw));
+  int* const cnt_rb = const_cast<int*>(flags + 16);         // [rbl] the CTA's units of it
   int* const done_rb = cnt_rb + kNrMaxRbl;                  // [rbl] of those, finished
-  // order[i] of the CTA's units in processing order: rbl | j << 8 | t << 16
-  // (t = rank of j among the CTA's slice steps, the activation stage use);
-  // inv[rbl * kNrMaxJ + j] = i; jsel[t] = j
-  int* const order = reinterpret_cast<int*>(smem_raw + (bars + kNrBarBytes - raw));
+  // order[i] of the CTA's units in processing order: rbl | j << 8;
+  // inv[rbl * kNrMaxJ + j] = i
+  int* const order = reinterpret_cast<int*>(smem_raw + (fl + kNrBarBytes - raw));
   int* const inv = order + kNrMaxUnits;
-  int* const jsel = inv + kNrMaxRbl * kNrMaxJ;
   uint32_t* const tblw = reinterpret_cast<uint32_t*>(gbase + p.tbl_off);
   float* const slot_f = reinterpret_cast<float*>(gbase + p.slot_off);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const uint64_t tmo = p.timeout_ns;
+  const int g = lane >> 2, c = lane & 3;
   const int cta = blockIdx.x;
   const int u0 = nr_begin(p.U, p.P, cta), u1 = nr_begin(p.U, p.P, cta + 1);
   const int n_units = u1 - u0;
@@ -312,60 +323,29 @@ __global__ void __launch_bounds__(kNrThreads, 1)
   if (tid == 0) {
     NR_STAMP(0);
     griddep_launch_dependents();
-    for (int s = 0; s < p.CS; ++s) {
-      mbar_init(bar_cfull + 8 * s, 1);
-      mbar_init(bar_cempty + 8 * s, 1);
-      ctag[s] = -1;
-    }
-    for (int s = 0; s < p.XS; ++s) {
-      mbar_init(bar_xfull + 8 * s, 1);
-      mbar_init(bar_xempty + 8 * s, kNrMaxRbl);
-      xtag[s] = -1;
-    }
     int bad = 0;
     if (n_units < 1 || n_units > p.max_units || n_units > kNrMaxUnits || n_rbl > p.max_rbl ||
-        n_rbl > kNrMaxRbl || p.Q > kNrMaxJ || p.CS > kNrMaxCS || p.XS > kNrMaxXS || p.CS < 1 ||
-        p.XS < 1 || p.M < 1 || p.M > MT)
+        n_rbl > kNrMaxRbl || p.Q > kNrMaxJ || p.M < 1 || p.M > MT)
       bad = 40;
-    // slice steps present in this CTA, in order: their rank is the
-    // activation stage use
-    int t = 0;
-    int jrank[kNrMaxJ];
-    for (int j = 0; j < p.Q && !bad; ++j) {
-      bool any = false;
-      for (int rbl = 0; rbl < n_rbl; ++rbl) {
-        const int u = (rb_lo + rbl) * p.Q + j;
-        any = any || (u >= u0 && u < u1);
-      }
-      jrank[j] = any ? t : -1;
-      if (any) jsel[t++] = j;
-    }
-    if (p.resident_x && t > p.XS) bad = 44;
+    // processing order: row block by row block (a row block shared with the
+    // previous CTA comes first and is finished early)
+    int i = 0;
     for (int rbl = 0; rbl < n_rbl && !bad; ++rbl) {
       cnt_rb[rbl] = 0;
       done_rb[rbl] = 0;
-    }
-    // processing order: with every activation stage resident, row block by
-    // row block (a row block shared with the previous CTA comes first and
-    // is finished early); else slice step by slice step
-    int i = 0;
-    for (int a = 0; a < (p.resident_x ? n_rbl : p.Q) && !bad; ++a) {
-      for (int b = 0; b < (p.resident_x ? p.Q : n_rbl); ++b) {
-        const int rbl = p.resident_x ? a : b, j = p.resident_x ? b : a;
+      for (int j = 0; j < p.Q; ++j) {
         const int u = (rb_lo + rbl) * p.Q + j;
         if (u >= u0 && u < u1) {
           inv[rbl * kNrMaxJ + j] = i;
-          order[i++] = rbl | (j << 8) | (jrank[j] << 16);
+          order[i++] = rbl | (j << 8);
           ++cnt_rb[rbl];
         }
       }
     }
     if (!bad && i != n_units) bad = 41;
     flags[0] = bad;
-    flags[1] = t;          // slice steps of this CTA
     flags[2] = 0;          // abort: a bounded wait gave up
     if (bad) atomicCAS(&g_device_error, 0, bad);
-    fence_mbar_init();
   }
   __syncthreads();
   // programmatic dependent launch: nothing written by the preceding grid is
@@ -373,89 +353,72 @@ __global__ void __launch_bounds__(kNrThreads, 1)
   griddep_wait();
   if (tid == 0) NR_STAMP(4);
   if (flags[0]) return;
-  const int n_j = flags[1];
 
-  int issued_c = 0, issued_x = 0;           // producer: copies issued so far
-  if (warp == kNrProducerWarp) {
-    // ---------------------------------------------------------- producer
-    if (lane == 0) {
-      prefetch_tensormap(&wmap);
-      prefetch_tensormap(&xmap);
-      bool ok = true;
-      if (p.resident_x) {
-        // every slice step's activations, once
-        for (int t = 0; t < n_j; ++t) {
-          xtag[t] = t;
-          mbar_arrive_expect_tx(bar_xfull + 8 * t, static_cast<uint32_t>(p.M) * 1024u);
-          tma_load_4d(xs0 + t * p.M * 1024, &xmap, 0, 0, 0, jsel[t] * 16, bar_xfull + 8 * t);
-          ++issued_x;
-        }
-      }
-      int t_next = 0;                       // ring mode: next activation use to load
-      for (int i = 0; i < n_units && ok; ++i) {
-        const int ord = order[i];
-        const int rbl = ord & 255, j = (ord >> 8) & 255, t = ord >> 16;
-        if (!p.resident_x && t == t_next) {
-          // the activation stage of slice step j: the units of this step release it
-          const int xs = t % p.XS;
-          if (!gv_wait(bar_xempty + 8 * xs, ((t / p.XS) & 1) ^ 1, flags + 2, tmo,
-                       SITE_NR_XEMPTY)) {
-            ok = false;
-            break;
-          }
-          int cnt = 0;
-          for (int r = 0; r < n_rbl; ++r) {
-            const int u = (rb_lo + r) * p.Q + j;
-            cnt += (u >= u0 && u < u1) ? 1 : 0;
-          }
-          // arrivals of the units that will not use this stage
-          if (kNrMaxRbl - cnt > 0) mbar_arrive_cnt(bar_xempty + 8 * xs, kNrMaxRbl - cnt);
-          xtag[xs] = t;
-          mbar_arrive_expect_tx(bar_xfull + 8 * xs, static_cast<uint32_t>(p.M) * 1024u);
-          tma_load_4d(xs0 + xs * p.M * 1024, &xmap, 0, 0, 0, j * 16, bar_xfull + 8 * xs);
-          ++t_next;
-          ++issued_x;
-        }
-        const int cs = i % p.CS;
-        if (!gv_wait(bar_cempty + 8 * cs, ((i / p.CS) & 1) ^ 1, flags + 2, tmo,
-                     SITE_NR_CEMPTY)) {
-          ok = false;
-          break;
-        }
-        ctag[cs] = i;
-        mbar_arrive_expect_tx(bar_cfull + 8 * cs, static_cast<uint32_t>(C::STAGE));
-        const int rb = rb_lo + rbl;
-        if (p.epilogue == CQ_EPI_SWIGLU)
-          tma_load_4d(codes0 + cs * C::STAGE, &wmap, j * C::SLICE, 0, rb * 8, 0,
-                      bar_cfull + 8 * cs);
-        else
-          tma_load_3d(codes0 + cs * C::STAGE, &wmap, j * C::SLICE, 0, rb * 16,
-                      bar_cfull + 8 * cs);
-        ++issued_c;
+  // -------------------------------------------------------- level tables
+  // block (rbl, it, lgi) holds the tables of lanes (g, c) = rows (rb, it, g)
+  // x groups (first group of quarter c) + lgi, entry e of lane l at word
+  // (block * E + e) * 32 + l.  The group parameters go out first, before
+  // the bulk of the loads, so that the tables are not held up behind them.
+    const int n_items = n_rbl * 2 * p.L * 32;
+    float s_pre[kNrPreItems];
+    uint32_t ab_pre[kNrPreItems];
+#pragma unroll
+    for (int k = 0; k < kNrPreItems; ++k) {
+      s_pre[k] = 0.f;
+      ab_pre[k] = 0u;
+      const int id = tid + k * kNrThreads;
+      int row, grp;
+      if (id < n_items && nr_item(p, rb_lo, id, row, grp)) {
+        const int64_t mi = static_cast<int64_t>(row) * p.ng + grp;
+        s_pre[k] = __uint_as_float(ldg_u32_ordered(p.scales + mi));
+        ab_pre[k] = ldg_u32_ordered(p.ab + mi);
       }
     }
-    __syncwarp();
-  } else {
-    // ---------------------------------------------------------- compute warps
-    // level tables: block (rbl, it, lgi) holds the tables of lanes (g, c) =
-    // rows (rb, it, g) x groups (first group of quarter c) + lgi, entry e of
-    // lane l at word (block * E + e) * 32 + l
-    const int n_items = n_rbl * 2 * p.L * 32;
-    for (int id = tid; id < n_items; id += kNrCompute * 32) {
+
+  // -------------------------------------------- loads: activations, codes
+  // every slice step's activations, as 16-byte chunks (j, s'', m, c)
+  {
+    const int n_chunks = p.Q * 16 * p.M * 4;
+    for (int ch = tid; ch < n_chunks; ch += kNrThreads) {
+      const int cq = ch & 3;
+      const int m = (ch >> 2) % p.M;
+      const int js = (ch >> 2) / p.M;                   // j * 16 + s''
+      const int j = js >> 4, s2 = js & 15;
+      const uint16_t* src =
+          p.x + static_cast<int64_t>(m) * p.K + cq * (p.K / 4) + j * 128 + s2 * 8;
+      cp_async16(xs0 + ch * 16, src);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  // codes of this warp's first units (registers)
+  uint32_t cn0[NB][4 * B], cn1[NB][4 * B];
+#pragma unroll
+  for (int k = 0; k < NB; ++k) {
+    const int i = warp + k * kNrCompute;
+#pragma unroll
+    for (int w = 0; w < 4 * B; ++w) cn0[k][w] = cn1[k][w] = 0u;
+    if (i < n_units) {
+      const int ord = order[i];
+      nr_load_codes<B>(p, rb_lo + (ord & 255), ord >> 8, g, c, cn0[k], cn1[k]);
+    }
+  }
+
+  {
+    for (int k = 0, id = tid; id < n_items; ++k, id += kNrThreads) {
       const int ln = id & 31;
       const int blk = id >> 5;
-      const int lgi = blk % p.L;
-      const int it = (blk / p.L) & 1;
-      const int rbl = blk / (2 * p.L);
-      const int g = ln >> 2, c = ln & 3;
-      const int rb = rb_lo + rbl;
-      const int row = gv_row(p.N, p.epilogue, rb, it, g);
-      const int grp = (c * p.Q) / p.spc + lgi;
-      const int grp_last = ((c + 1) * p.Q - 1) / p.spc;
-      const bool valid = row < p.N && grp <= grp_last && grp < p.ng && rb < p.n_rb;
+      int row, grp;
+      const bool valid = nr_item(p, rb_lo, id, row, grp);
       float s = 0.f;
       uint32_t abw = 0u;
-      if (valid) {
+      if (k < kNrPreItems) {
+#pragma unroll
+        for (int kk = 0; kk < kNrPreItems; ++kk)
+          if (kk == k) {
+            s = s_pre[kk];
+            abw = ab_pre[kk];
+          }
+      } else if (valid) {
         const int64_t mi = static_cast<int64_t>(row) * p.ng + grp;
         s = __ldg(p.scales + mi);
         abw = __ldg(p.ab + mi);
@@ -472,145 +435,128 @@ __global__ void __launch_bounds__(kNrThreads, 1)
         for (int e = 0; e < E; ++e) tb[e * 32] = Lv[e & (NL - 1)] | (Lv[e / NL] << 16);
       }
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kNrCompute * 32) : "memory");
-    if (tid == 0) NR_STAMP(2);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  if (tid == 0) NR_STAMP(2);
 
-    const int g = lane >> 2, c = lane & 3;
-    // 16-byte chunk order of the code reads (keeps them conflict free)
-    const int rot = B == 2 ? (g & 1) : (B == 4 ? (g & 1) + 2 * (c >> 1) : 0);
-    long long cyc_wait = 0, cyc_work = 0, cyc_fin = 0;
-    bool ok = true;
-    for (int i = warp; i < n_units && ok; i += kNrCompute) {
-      const long long t_a = p.trace ? clock64() : 0;
-      const int ord = order[i];
-      const int rbl = ord & 255, j = (ord >> 8) & 255, t = ord >> 16;
-      const int cs = i % p.CS, xs = t % p.XS;
-      const bool tag_ok = nr_wait_tag(ctag + cs, i, flags + 2, tmo, SITE_NR_CFULL);
-      if (!__all_sync(0xffffffffu, tag_ok) ||
-          !gv_wait_warp(bar_cfull + 8 * cs, (i / p.CS) & 1, flags + 2, tmo, SITE_NR_CFULL)) {
-        ok = false;
-        break;
+  // ------------------------------------------------------------ the units
+  long long cyc_work = 0, cyc_fin = 0;
+  bool ok = true;
+  for (int i = warp; i < n_units && ok; i += kNrCompute) {
+    const long long t_a = p.trace ? clock64() : 0;
+    const int ord = order[i];
+    const int rbl = ord & 255, j = ord >> 8;
+    // this unit's codes; the warp's unit NB ahead goes into the freed buffer
+    uint32_t c0[4 * B], c1[4 * B];
+#pragma unroll
+    for (int w = 0; w < 4 * B; ++w) {
+      c0[w] = cn0[0][w];
+      c1[w] = cn1[0][w];
+    }
+#pragma unroll
+    for (int kb = 0; kb + 1 < NB; ++kb)
+#pragma unroll
+      for (int w = 0; w < 4 * B; ++w) {
+        cn0[kb][w] = cn0[kb + 1][w];
+        cn1[kb][w] = cn1[kb + 1][w];
       }
-      // the lane's two rows (g, g+8) of slice j of quarter c
-      const uint32_t cb = codes0 + cs * C::STAGE + (g * 4 + c) * C::SLICE;
-      uint32_t c0[4 * B], c1[4 * B];
-#pragma unroll
-      for (int v = 0; v < B; ++v) {
-        int vv = v + rot;
-        while (vv >= B) vv -= B;
-        const uint4 q0 = lds128(cb + 16 * vv);
-        const uint4 q1 = lds128(cb + 32 * C::SLICE + 16 * vv);
-#pragma unroll
-        for (int w = 0; w < B; ++w)
-          if (w == vv) {
-            c0[4 * w + 0] = q0.x;
-            c0[4 * w + 1] = q0.y;
-            c0[4 * w + 2] = q0.z;
-            c0[4 * w + 3] = q0.w;
-            c1[4 * w + 0] = q1.x;
-            c1[4 * w + 1] = q1.y;
-            c1[4 * w + 2] = q1.z;
-            c1[4 * w + 3] = q1.w;
-          }
+    {
+      const int ia = i + NB * kNrCompute;
+      if (ia < n_units) {
+        const int oa = order[ia];
+        nr_load_codes<B>(p, rb_lo + (oa & 255), oa >> 8, g, c, cn0[NB - 1], cn1[NB - 1]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_cempty + 8 * cs);
-      const bool xtag_ok = nr_wait_tag(xtag + xs, t, flags + 2, tmo, SITE_NR_XFULL);
-      if (!__all_sync(0xffffffffu, xtag_ok) ||
-          !gv_wait_warp(bar_xfull + 8 * xs, (t / p.XS) & 1, flags + 2, tmo, SITE_NR_XFULL)) {
-        ok = false;
-        break;
-      }
-      const long long t_b = p.trace ? clock64() : 0;
-      const int lgi = nr_lgi(p.Q, p.spc, c, j);
-      const uint32_t blk0 = static_cast<uint32_t>(((rbl * 2 + 0) * p.L + lgi) * E * 128);
-      const uint32_t blk1 = static_cast<uint32_t>(((rbl * 2 + 1) * p.L + lgi) * E * 128);
-      const uint32_t tl0 = tbl0 + blk0 + lane * 4;
-      const uint32_t tl1 = tbl0 + blk1 + lane * 4;
-      // activations: [k pair s''][token][quarter][8 values]
-      const uint32_t xa = xs0 + xs * p.M * 1024 + (g * 4 + c) * 16;
-      const uint32_t xstride = static_cast<uint32_t>(p.M) * 64u;
-      const bool xl0 = g < p.M;
-      const bool xl1 = MT == 16 && g + 8 < p.M;
-      float acc[2][MT / 8][4];
+    }
+    const int lgi = nr_lgi(p.Q, p.spc, c, j);
+    const uint32_t blk0 = static_cast<uint32_t>(((rbl * 2 + 0) * p.L + lgi) * E * 128);
+    const uint32_t blk1 = static_cast<uint32_t>(((rbl * 2 + 1) * p.L + lgi) * E * 128);
+    const uint32_t tl0 = tbl0 + blk0 + lane * 4;
+    const uint32_t tl1 = tbl0 + blk1 + lane * 4;
+    // activations: [j][k pair s''][token][quarter][8 values]
+    const uint32_t xa = xs0 + j * p.M * 1024 + (g * 4 + c) * 16;
+    const uint32_t xstride = static_cast<uint32_t>(p.M) * 64u;
+    const bool xl0 = g < p.M;
+    const bool xl1 = MT == 16 && g + 8 < p.M;
+    float acc[2][MT / 8][4];
 #pragma unroll
-      for (int a = 0; a < 2; ++a)
-#pragma unroll
-        for (int h = 0; h < MT / 8; ++h)
-#pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][h][b] = 0.f;
-      uint4 xv0 = make_uint4(0u, 0u, 0u, 0u), xv1 = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2) {
-        if (xl0) xv0 = lds128(xa + s2 * xstride);
-        if (MT == 16 && xl1) xv1 = lds128(xa + s2 * xstride + 8 * 64);
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int s = 2 * s2 + h2;          // MMA step: codes 4s .. 4s+3
-          const uint32_t a0 = gv_pair<B>(c0, 2 * s, tl0);
-          const uint32_t a1 = gv_pair<B>(c1, 2 * s, tl1);
-          const uint32_t a2 = gv_pair<B>(c0, 2 * s + 1, tl0);
-          const uint32_t a3 = gv_pair<B>(c1, 2 * s + 1, tl1);
-          const uint32_t b0 = h2 ? xv0.z : xv0.x, b1 = h2 ? xv0.w : xv0.y;
-          mma_16816_bf16(acc[h2][0], a0, a1, a2, a3, b0, b1);
-          if constexpr (MT == 16) {
-            const uint32_t e0 = h2 ? xv1.z : xv1.x, e1 = h2 ? xv1.w : xv1.y;
-            mma_16816_bf16(acc[h2][1], a0, a1, a2, a3, e0, e1);
-          }
-        }
-      }
-      __syncwarp();
-      if (!p.resident_x && lane == 0) mbar_arrive(bar_xempty + 8 * xs);
-      // the unit's partial sums: [unit][lane][NV]
-      float* const sl = slot_f + (i * 32 + lane) * NV;
+    for (int a = 0; a < 2; ++a)
 #pragma unroll
       for (int h = 0; h < MT / 8; ++h)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) sl[h * 4 + b] = acc[0][h][b] + acc[1][h][b];
-      // the warp that finishes a row block's last unit in this CTA sums it
+        for (int b = 0; b < 4; ++b) acc[a][h][b] = 0.f;
+    // software-pipelined: the lookups of MMA step s+2 and the activations of
+    // the next k pair are issued before the MMA of step s
+    uint4 xv0 = make_uint4(0u, 0u, 0u, 0u), xv1 = make_uint4(0u, 0u, 0u, 0u);
+    uint4 xn0 = xv0, xn1 = xv1;
+    if (xl0) xv0 = lds128(xa);
+    if (MT == 16 && xl1) xv1 = lds128(xa + 8 * 64);
+    uint32_t a[3][4];
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      a[s][0] = gv_pair<B>(c0, 2 * s, tl0);
+      a[s][1] = gv_pair<B>(c1, 2 * s, tl1);
+      a[s][2] = gv_pair<B>(c0, 2 * s + 1, tl0);
+      a[s][3] = gv_pair<B>(c1, 2 * s + 1, tl1);
+    }
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2) {
+      if (s2 + 1 < 16) {
+        if (xl0) xn0 = lds128(xa + (s2 + 1) * xstride);
+        if (MT == 16 && xl1) xn1 = lds128(xa + (s2 + 1) * xstride + 8 * 64);
+      }
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int s = 2 * s2 + h2;          // MMA step: codes 4s .. 4s+3
+        if (s + 2 < 32) {
+          const int sn = s + 2;
+          a[sn % 3][0] = gv_pair<B>(c0, 2 * sn, tl0);
+          a[sn % 3][1] = gv_pair<B>(c1, 2 * sn, tl1);
+          a[sn % 3][2] = gv_pair<B>(c0, 2 * sn + 1, tl0);
+          a[sn % 3][3] = gv_pair<B>(c1, 2 * sn + 1, tl1);
+        }
+        const uint32_t* as = a[s % 3];
+        const uint32_t b0 = h2 ? xv0.z : xv0.x, b1 = h2 ? xv0.w : xv0.y;
+        mma_16816_bf16(acc[h2][0], as[0], as[1], as[2], as[3], b0, b1);
+        if constexpr (MT == 16) {
+          const uint32_t e0 = h2 ? xv1.z : xv1.x, e1 = h2 ? xv1.w : xv1.y;
+          mma_16816_bf16(acc[h2][1], as[0], as[1], as[2], as[3], e0, e1);
+        }
+      }
+      xv0 = xn0;
+      xv1 = xn1;
+    }
+    // the unit's partial sums: [unit][lane][NV]
+    float* const sl = slot_f + (i * 32 + lane) * NV;
+#pragma unroll
+    for (int h = 0; h < MT / 8; ++h)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) sl[h * 4 + b] = acc[0][h][b] + acc[1][h][b];
+    // the warp that finishes a row block's last unit in this CTA sums it
+    __threadfence_block();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) last = atomicAdd(done_rb + rbl, 1) + 1 == cnt_rb[rbl];
+    last = __shfl_sync(0xffffffffu, last, 0);
+    const long long t_c = p.trace ? clock64() : 0;
+    if (last) {
       __threadfence_block();
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) last = atomicAdd(done_rb + rbl, 1) + 1 == cnt_rb[rbl];
-      last = __shfl_sync(0xffffffffu, last, 0);
-      const long long t_c = p.trace ? clock64() : 0;
-      if (last) {
-        __threadfence_block();
-        if (!nr_finish_row_block<MT>(p, cta, rb_lo + rbl, u0, u1, rbl, inv, slot_f, lane,
-                                     flags + 2))
-          ok = false;
-      }
-      if (p.trace) {
-        const long long t_d = clock64();
-        cyc_wait += t_b - t_a;
-        cyc_work += t_c - t_b;
-        cyc_fin += t_d - t_c;
-      }
+      if (!nr_finish_row_block<MT>(p, cta, rb_lo + rbl, u0, u1, rbl, inv, slot_f, lane,
+                                   flags + 2))
+        ok = false;
     }
-    if (p.trace && lane == 0) {
-      p.trace[blockIdx.x * 64 + 8 + 3 * warp] = cyc_wait;
-      p.trace[blockIdx.x * 64 + 9 + 3 * warp] = cyc_work;
-      p.trace[blockIdx.x * 64 + 10 + 3 * warp] = cyc_fin;
+    if (p.trace) {
+      cyc_work += t_c - t_a;
+      cyc_fin += clock64() - t_c;
     }
+  }
+  if (p.trace && lane == 0) {
+    p.trace[blockIdx.x * 64 + 8 + 3 * warp] = 0;
+    p.trace[blockIdx.x * 64 + 9 + 3 * warp] = cyc_work;
+    p.trace[blockIdx.x * 64 + 10 + 3 * warp] = cyc_fin;
   }
   __syncthreads();
   if (tid == 0) NR_STAMP(1);
-  if (flags[2]) {
-    // a wait gave up: no copy may still be landing in shared memory at exit
-    if (warp == kNrProducerWarp && lane == 0) {
-      volatile int dummy = 0;
-      for (int k = 1; k <= issued_c && k <= p.CS; ++k) {
-        const int i = issued_c - k;
-        mbar_wait(bar_cfull + 8 * (i % p.CS), (i / p.CS) & 1, &dummy, tmo, SITE_TEARDOWN);
-      }
-      const int xk = p.resident_x ? issued_x : (issued_x < p.XS ? issued_x : p.XS);
-      for (int k = 1; k <= xk; ++k) {
-        const int t = issued_x - k;
-        mbar_wait(bar_xfull + 8 * (t % p.XS), (t / p.XS) & 1, &dummy, tmo, SITE_TEARDOWN);
-      }
-    }
-    __syncthreads();
-  }
 }
 
 }  // namespace cq

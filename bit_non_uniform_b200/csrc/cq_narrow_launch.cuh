@@ -1,6 +1,5 @@
 // cq_narrow_launch.cuh -- host side of the narrow-row GEMM (M <= 16): the
-// plan (units, CTA shares, ring depths, shared-memory layout), the tensor
-// maps over the packed matrix and the activations, and the launch with
+// plan (units, CTA shares, shared-memory layout) and the launch with
 // programmatic dependent launch.  Part of the single translation unit of
 // libcq (included by cq_gemm.cu).
 #pragma once
@@ -16,8 +15,8 @@ namespace cq {
 
 struct NrPlan {
   bool use;
-  int MT, n_rb, Q, spc, ng, L, U, P, max_units, max_rbl, CS, XS, resident_x;
-  int tbl_off, code_off, x_off, slot_off, smem;
+  int MT, n_rb, Q, spc, ng, L, U, P, max_units, max_rbl;
+  int tbl_off, x_off, slot_off, smem;
   size_t ws_counter_bytes, ws_partial_bytes;
 };
 
@@ -53,101 +52,27 @@ static NrPlan plan_narrow(int64_t M, int64_t N, int64_t K, int B, int G, int epi
   if (v.max_units > kNrMaxUnits || v.max_rbl > kNrMaxRbl) return v;
   const int E = B == 3 ? 64 : 16;
   const int tbl_bytes = v.max_rbl * 2 * v.L * E * 128;
-  const int code_stage = 1024 * B;
-  const int x_stage = 1024 * static_cast<int>(M);
+  const int64_t x_bytes = M * K * 2;              // every slice step of every token
   const int slot_bytes = 512 * (v.MT / 8);
-  auto align = [](int x, int a) { return (x + a - 1) / a * a; };
-  auto layout = [&](int CS, int XS) {
-    v.CS = CS;
-    v.XS = XS;
-    v.tbl_off = 0;
-    v.code_off = align(tbl_bytes, 1024);
-    v.x_off = align(v.code_off + CS * code_stage, 1024);
-    v.slot_off = align(v.x_off + XS * x_stage, 128);
-    // the table base is aligned up to a table block (E * 128 bytes) from the
-    // 16-byte aligned start of the dynamic shared memory
-    v.smem = E * 128 + v.slot_off + v.max_units * slot_bytes + kNrBarBytes + kNrOrderBytes;
-    return v.smem <= 227 * 1024;
-  };
-  // preferred: every slice step's activations resident and every unit's codes
-  // in flight at once; then fewer code stages; then an activation ring
-  const int cs_all = v.max_units < kNrMaxCS ? v.max_units : kNrMaxCS;
-  bool fits = false;
-  if (v.Q <= kNrMaxXS) {
-    v.resident_x = 1;
-    for (int CS = cs_all; CS >= 1 && !fits; CS = CS > 8 ? CS - 4 : CS - 1)
-      fits = layout(CS, v.Q);
-  }
-  if (!fits) {
-    v.resident_x = 0;
-    const int xs0 = v.Q < 4 ? v.Q : 4;
-    for (int XS = xs0; XS >= 2 && !fits; --XS)
-      for (int CS = cs_all; CS >= 1 && !fits; CS = CS > 8 ? CS - 4 : CS - 1)
-        fits = layout(CS, XS);
-  }
-  if (!fits) return v;
+  v.tbl_off = 0;
+  v.x_off = (tbl_bytes + 1023) / 1024 * 1024;
+  const int64_t slot_off = (v.x_off + x_bytes + 127) / 128 * 128;
+  // the table base is aligned up to a table block (E * 128 bytes) from the
+  // 16-byte aligned start of the dynamic shared memory
+  const int64_t smem =
+      E * 128 + slot_off + static_cast<int64_t>(v.max_units) * slot_bytes + kNrBarBytes +
+      kNrOrderBytes;
+  if (smem > 227 * 1024) return v;
+  v.slot_off = static_cast<int>(slot_off);
+  v.smem = static_cast<int>(smem);
   v.ws_counter_bytes = (static_cast<size_t>(v.n_rb) * sizeof(int) + 255) / 256 * 256;
   v.ws_partial_bytes = static_cast<size_t>(v.P) * 16 * v.MT * sizeof(float);
   v.use = true;
   return v;
 }
 
-// Packed codes for the narrow kernel: one box = one slice (16*B bytes) of each
-// of the four quarters of 16 rows (SwiGLU: 8 gate rows and the 8 matching up
-// rows), landing in shared memory as [row][quarter][16*B bytes].
-static int encode_packed_narrow(CUtensorMap* map, const void* base, int64_t N, int64_t K, int B,
-                                int epilogue) {
-  EncodeTiledFn fn = encode_tiled_fn();
-  if (!fn) return CQ_ERR_CUDA;
-  const int64_t row_bytes = K * B / 8;
-  const int64_t quarter = row_bytes / 4;
-  const cuuint32_t slice = static_cast<cuuint32_t>(16 * B);
-  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-  CUresult r;
-  if (epilogue == CQ_EPI_SWIGLU) {
-    cuuint64_t dims[4] = {static_cast<cuuint64_t>(quarter), 4u,
-                          static_cast<cuuint64_t>(N / 2), 2u};
-    cuuint64_t strides[3] = {static_cast<cuuint64_t>(quarter),
-                             static_cast<cuuint64_t>(row_bytes),
-                             static_cast<cuuint64_t>((N / 2) * row_bytes)};
-    cuuint32_t box[4] = {slice, 4u, 8u, 2u};
-    r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box,
-           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  } else {
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(quarter), 4u, static_cast<cuuint64_t>(N)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(quarter),
-                             static_cast<cuuint64_t>(row_bytes)};
-    cuuint32_t box[3] = {slice, 4u, 16u};
-    r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
-           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  }
-  return r == CUDA_SUCCESS ? CQ_OK : CQ_ERR_CUDA;
-}
-
-// Activations for the narrow kernel, bf16 [M][K] viewed as 4-D
-//   (8 values [16 bytes], quarter [stride K/4 values], token [stride K],
-//    8-value chunk within the quarter [stride 8 values]);
-// one box = the 16 chunks of one slice step of all tokens and quarters,
-// landing as [chunk][token][quarter][8 values].
-static int encode_x_narrow(CUtensorMap* map, const void* x, int64_t M, int64_t K) {
-  EncodeTiledFn fn = encode_tiled_fn();
-  if (!fn) return CQ_ERR_CUDA;
-  cuuint64_t dims[4] = {8u, 4u, static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(K / 32)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(K / 4 * 2), static_cast<cuuint64_t>(K * 2),
-                           16u};
-  cuuint32_t box[4] = {8u, 4u, static_cast<cuuint32_t>(M), 16u};
-  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? CQ_OK : CQ_ERR_CUDA;
-}
-
 template <int B, int MT>
-static int launch_narrow(const NarrowParams& p, const CUtensorMap& wmap, const CUtensorMap& xmap,
-                         cudaStream_t s) {
+static int launch_narrow(const NarrowParams& p, cudaStream_t s) {
   static std::atomic<uint64_t> smem_set{0};
   if (!ensure_smem_limit(narrow_kernel<B, MT>, 227 * 1024, smem_set)) return CQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
@@ -160,7 +85,7 @@ static int launch_narrow(const NarrowParams& p, const CUtensorMap& wmap, const C
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, narrow_kernel<B, MT>, p, wmap, xmap) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, narrow_kernel<B, MT>, p) != cudaSuccess)
     return CQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
 }
@@ -170,11 +95,6 @@ static int run_narrow(const NrPlan& v, const uint16_t* x, int64_t M, const uint8
                       int G, int grid_mode, int epilogue, int out_dtype, void* y,
                       void* workspace, cudaStream_t stream, uint64_t timeout_ns,
                       uint64_t* trace) {
-  CUtensorMap wmap, xmap;
-  int st = encode_packed_narrow(&wmap, packed, N, K, B, epilogue);
-  if (st != CQ_OK) return st;
-  st = encode_x_narrow(&xmap, x, M, K);
-  if (st != CQ_OK) return st;
   NarrowParams p = {};
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
@@ -192,16 +112,15 @@ static int run_narrow(const NrPlan& v, const uint16_t* x, int64_t M, const uint8
   p.P = v.P;
   p.max_rbl = v.max_rbl;
   p.max_units = v.max_units;
-  p.CS = v.CS;
-  p.XS = v.XS;
-  p.resident_x = v.resident_x;
   p.tbl_off = v.tbl_off;
-  p.code_off = v.code_off;
   p.x_off = v.x_off;
   p.slot_off = v.slot_off;
   p.smem_bytes = v.smem;
+  p.packed = packed;
+  p.row_bytes = K * B / 8;
   p.scales = scales;
   p.ab = reinterpret_cast<const uint32_t*>(ab);
+  p.x = x;
   p.y = y;
   p.ldy = epilogue == CQ_EPI_SWIGLU ? N / 2 : N;
   p.counter = reinterpret_cast<int*>(workspace);
@@ -212,13 +131,13 @@ static int run_narrow(const NrPlan& v, const uint16_t* x, int64_t M, const uint8
   p.timeout_ns = timeout_ns;
   p.trace = reinterpret_cast<unsigned long long*>(trace);
   if (v.MT == 8) {
-    if (B == 2) return launch_narrow<2, 8>(p, wmap, xmap, stream);
-    if (B == 3) return launch_narrow<3, 8>(p, wmap, xmap, stream);
-    return launch_narrow<4, 8>(p, wmap, xmap, stream);
+    if (B == 2) return launch_narrow<2, 8>(p, stream);
+    if (B == 3) return launch_narrow<3, 8>(p, stream);
+    return launch_narrow<4, 8>(p, stream);
   }
-  if (B == 2) return launch_narrow<2, 16>(p, wmap, xmap, stream);
-  if (B == 3) return launch_narrow<3, 16>(p, wmap, xmap, stream);
-  return launch_narrow<4, 16>(p, wmap, xmap, stream);
+  if (B == 2) return launch_narrow<2, 16>(p, stream);
+  if (B == 3) return launch_narrow<3, 16>(p, stream);
+  return launch_narrow<4, 16>(p, stream);
 }
 
 }  // namespace cq
