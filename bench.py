@@ -39,25 +39,39 @@ import torch  # noqa: E402
 
 METRIC = "Cubic GEMM packed-weight GB/s at M=1 and TFLOP/s at M>=256, % of B200 roofline"
 
+_DOWN = "Kimi-K3 expert down_proj, CubicQuant W3 G512, N=7168 x K=3072"
+_GU = "Kimi-K3 expert gate+up, CubicQuant W2 G512, N=6144 x K=7168, SwiGLU"
 WORKLOADS = {
     # name: (description, N, K, B, G, M, epilogue)
-    "down_m1": ("Kimi-K3 expert down_proj, CubicQuant W3 G512, N=7168 x K=3072, M=1",
-                7168, 3072, 3, 512, 1, 0),
-    "gate_up_m1": ("Kimi-K3 expert gate+up, CubicQuant W2 G512, N=6144 x K=7168, M=1, SwiGLU",
-                   6144, 7168, 2, 512, 1, 1),
-    "down_m16": ("Kimi-K3 expert down_proj, W3 G512, N=7168 x K=3072, M=16",
-                 7168, 3072, 3, 512, 16, 0),
-    "gate_up_m4096": ("Kimi-K3 expert gate+up, W2 G512, N=6144 x K=7168, M=4096, SwiGLU",
-                      6144, 7168, 2, 512, 4096, 1),
-    "down_m4096": ("Kimi-K3 expert down_proj, W3 G512, N=7168 x K=3072, M=4096",
-                   7168, 3072, 3, 512, 4096, 0),
+    "down_m1": (f"{_DOWN}, M=1", 7168, 3072, 3, 512, 1, 0),
+    "down_m4": (f"{_DOWN}, M=4", 7168, 3072, 3, 512, 4, 0),
+    "down_m16": (f"{_DOWN}, M=16", 7168, 3072, 3, 512, 16, 0),
+    "gate_up_m1": (f"{_GU}, M=1", 6144, 7168, 2, 512, 1, 1),
+    "gate_up_m16": (f"{_GU}, M=16", 6144, 7168, 2, 512, 16, 1),
+    "gate_up_m64": (f"{_GU}, M=64", 6144, 7168, 2, 512, 64, 1),
+    # the M >= 256 clause of the metric on single-matrix shapes (an extension of
+    # the configurations: same matrices, larger token counts)
+    "down_m256": (f"{_DOWN}, M=256", 7168, 3072, 3, 512, 256, 0),
+    "gate_up_m1024": (f"{_GU}, M=1024", 6144, 7168, 2, 512, 1024, 1),
+    "gate_up_m4096": (f"{_GU}, M=4096", 6144, 7168, 2, 512, 4096, 1),
+    "down_m4096": (f"{_DOWN}, M=4096", 7168, 3072, 3, 512, 4096, 0),
+    # the Dynamic A8 path (INT8 activations) beside A16, where the article
+    # reports the crossover ("实验结果 2. H200 内核交叉点")
+    "a8_gate_up_m64": (f"Dynamic A8: {_GU}, M=64", 6144, 7168, 2, 512, 64, 1),
+    "a8_down_m256": (f"Dynamic A8: {_DOWN}, M=256", 7168, 3072, 3, 512, 256, 0),
+    "a8_gate_up_m4096": (f"Dynamic A8: {_GU}, M=4096", 6144, 7168, 2, 512, 4096, 1),
 }
+# the GEMM lines printed under "secondary", in order
+SECONDARY = ["down_m4", "down_m16", "gate_up_m1", "gate_up_m16", "gate_up_m64", "down_m256",
+             "gate_up_m1024", "gate_up_m4096", "down_m4096", "a8_gate_up_m64", "a8_down_m256",
+             "a8_gate_up_m4096"]
+NOMINAL_HBM_GBS = 8000.0          # the ~8 TB/s HBM3e figure
+NOMINAL_BF16_TFLOPS = 2250.0      # dense BF16 datasheet figure
 
 
-# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture
-# (profiles/gemv_kernel_down_w3g512_m1.md).  Keyed by the SHA-256 of the kernel's
-# sources at capture time: once they change, the figure no longer describes the
-# kernel and `traffic` is reported as null.
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture.
+# Keyed by the SHA-256 of the kernel's sources at capture time: once they change,
+# the figure no longer describes the kernel and `traffic` is reported as null.
 KERNEL_SOURCES = ("cq_gemv.cuh", "cq_gemv_launch.cuh", "cq_device.cuh")
 TRAFFIC = {
     "down_m1": {"kernel": "gemv_kernel<3,1>", "bytes": 8652544,
@@ -97,8 +111,13 @@ def main_roofline(r, ach_gbs, hbm, tf_burst, traffic, name, peak_src):
 def dominant_kernel(name):
     """The kernel one cq_gemm launch of the workload runs (the only one it runs)."""
     _, N, K, B, G, M, epi = WORKLOADS[name]
+    if name.startswith("a8_"):
+        nt = 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
+        return f"quant_rows_kernel + engine_a8_kernel<{nt},{64 if B == 3 else 16}>"
     if M <= 2:
         return f"gemv_kernel<{B},{M}>"
+    if M <= 5 and K % 512 == 0:
+        return f"narrow_kernel<{B},8>"
     if M <= 128:
         nt = 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
     else:
@@ -247,7 +266,27 @@ def rotation_copies(nbytes, l2_bytes):
     return max(2, int(np.ceil(4.5 * l2_bytes / nbytes)))
 
 
-def time_gemm(cq, name, steps, warmup, world, device, sample_clocks=False):
+# Cycles of the spin kernel queued ahead of the first timing event: it keeps the
+# GPU busy while the host enqueues the graph replay, so the timed region holds the
+# launches only, whatever the host-side latency of the replay call (about 0.5 ms
+# at the 1.9 GHz clock; much longer than any enqueue).
+SPIN_CYCLES = 1_000_000
+
+
+def timed_replay(g, stream):
+    """Milliseconds of one replay of graph g, CUDA events on `stream`, with a
+    spin kernel queued ahead of the first event."""
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(SPIN_CYCLES)
+        ev0.record(stream)
+        g.replay()
+        ev1.record(stream)
+    ev1.synchronize()
+    return ev0.elapsed_time(ev1)
+
+
+def time_gemm(cq, name, steps, warmup, world, device, sample_clocks=False, repeats=0):
     """Device-timed K steps of one workload (CUDA graph of K launches)."""
     desc, N, K, B, G, M, epi = WORKLOADS[name]
     import synthetic
@@ -259,12 +298,20 @@ def time_gemm(cq, name, steps, warmup, world, device, sample_clocks=False):
     x = synthetic.activations(11, M, K).to(device)
     ncol = N // 2 if epi else N
     y = torch.empty((M, ncol), dtype=torch.float32, device=device)
-    ws = cq.gemm_workspace(M, N, K, B, G, epi, device)
+    a8 = name.startswith("a8_")
+    if a8:
+        n = cq.gemm_a8_workspace_size(M, N, K, B, G, epi)
+        ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+    else:
+        ws = cq.gemm_workspace(M, N, K, B, G, epi, device)
     stream = torch.cuda.Stream(device)
 
     def step(i, st):
         p, sc, a = copies[i % R]
-        cq.cq_gemm(x, p, sc, a, N, K, B, G, epilogue=epi, workspace=ws, out=y, stream=st)
+        if a8:
+            cq.cq_gemm_a8(x, p, sc, a, N, K, B, G, epilogue=epi, workspace=ws, out=y, stream=st)
+        else:
+            cq.cq_gemm(x, p, sc, a, N, K, B, G, epilogue=epi, workspace=ws, out=y, stream=st)
 
     with torch.cuda.stream(stream):
         for i in range(max(warmup, 3)):
@@ -279,18 +326,17 @@ def time_gemm(cq, name, steps, warmup, world, device, sample_clocks=False):
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(device.index if device.index is not None else 0)
     with sampler if sample_clocks else _null():
-        ev0.record(stream)
-        with torch.cuda.stream(stream):
-            g.replay()
-        ev1.record(stream)
-        ev1.synchronize()
+        ms = timed_replay(g, stream)
     torch.cuda.synchronize()
     barrier(world)
-    ms = ev0.elapsed_time(ev1)
     ms = max_over_ranks(ms, world)
+    reps = []
+    if repeats:
+        for _ in range(repeats):
+            reps.append(timed_replay(g, stream) / steps)
+        torch.cuda.synchronize()
     st, site = cq.device_error()
     if st != 0:
         raise RuntimeError(f"device wait timed out (site {site})")
@@ -302,7 +348,69 @@ def time_gemm(cq, name, steps, warmup, world, device, sample_clocks=False):
                tflops=flops * steps / (ms * 1e-3) / 1e12,
                alg_bytes=wbytes + M * K * 2 + M * ncol * 4,
                clocks=sampler.summary() if sample_clocks else None)
+    if reps:
+        res["rep_ms_per_step"] = sorted(reps)
     return res
+
+
+def gemm_entry(r, hbm, tf_burst, world):
+    """One secondary line: HBM roofline up to M = 64, BF16 tensor above."""
+    ent = {"workload": r["desc"], "ms_per_step": round(r["ms_per_step"], 6),
+           "packed_gbs": round(r["gbs"] * world, 1), "tflops": round(r["tflops"] * world, 2),
+           "kernel": dominant_kernel(r["name"]),
+           "l2": f"{r['R']} rotating weight copies ({r['rot_mb']:.0f} MB)"}
+    if "rep_ms_per_step" in r:
+        ent["best_ms_per_step"] = round(min(r["rep_ms_per_step"]), 6)
+        ent["median_ms_per_step"] = round(statistics.median(r["rep_ms_per_step"]), 6)
+    if r["M"] <= 64:
+        ach = r["alg_bytes"] / (r["ms_per_step"] * 1e-3) / 1e9
+        ent["roofline"] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
+                           "unit": "GB/s", "frac": round(ach / hbm, 4),
+                           "frac_nominal": round(ach / NOMINAL_HBM_GBS, 4)}
+    elif r["name"].startswith("a8_"):
+        # INT8 tensor peak: the measured BF16 peak times the nominal 2x ratio
+        pk = 2.0 * tf_burst
+        ent["roofline"] = {"bound": "tensor", "achieved": round(r["tflops"], 1),
+                           "peak": round(pk, 1), "unit": "TOP/s",
+                           "frac": round(r["tflops"] / pk, 4),
+                           "frac_nominal": round(r["tflops"] / (2 * NOMINAL_BF16_TFLOPS), 4),
+                           "peak_kind": "int8 = 2 x the measured bf16 peak"}
+    else:
+        ent["roofline"] = {"bound": "tensor", "achieved": round(r["tflops"], 1),
+                           "peak": tf_burst, "unit": "TFLOP/s",
+                           "frac": round(r["tflops"] / tf_burst, 4),
+                           "frac_nominal": round(r["tflops"] / NOMINAL_BF16_TFLOPS, 4)}
+    return ent
+
+
+def time_cold(cq, name, device):
+    """One launch on a cold cache: L2 flushed by writing a buffer larger than
+    it, the GPU idle, an ordinary (non-graph) call.  Reports the CUDA-event
+    time on the stream (launch latency on the device included) and the host
+    wall time of the call plus synchronisation."""
+    desc, N, K, B, G, M, epi = WORKLOADS[name]
+    import synthetic
+    packed, s, ab = build_weights(cq, name, device)
+    x = synthetic.activations(13, M, K).to(device)
+    y = torch.empty((M, N // 2 if epi else N), dtype=torch.float32, device=device)
+    ws = cq.gemm_workspace(M, N, K, B, G, epi, device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(int(2 * l2), dtype=torch.uint8, device=device)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        cq.cq_gemm(x, packed, s, ab, N, K, B, G, epilogue=epi, workspace=ws, out=y,
+                   stream=stream)        # module and first-call setup, not timed
+        flush.fill_(1)
+    stream.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    ev0.record(stream)
+    cq.cq_gemm(x, packed, s, ab, N, K, B, G, epilogue=epi, workspace=ws, out=y, stream=stream)
+    ev1.record(stream)
+    ev1.synchronize()
+    wall = time.perf_counter() - t0
+    return {"device_us": round(ev0.elapsed_time(ev1) * 1e3, 2), "host_wall_us": round(wall * 1e6, 1),
+            "l2_flushed_bytes": int(flush.numel())}
 
 
 MOE_WORKLOADS = {
@@ -359,13 +467,7 @@ def time_moe(cq, name, steps, device):
             step()
     g.replay()
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    with torch.cuda.stream(stream):
-        g.replay()
-    ev1.record(stream)
-    ev1.synchronize()
-    ms = ev0.elapsed_time(ev1) / steps
+    ms = timed_replay(g, stream) / steps
     st, site = cq.device_error()
     if st != 0:
         raise RuntimeError(f"device wait timed out (site {site})")
@@ -444,13 +546,13 @@ def oracle_sample(name, rows):
             rows, K, B, G)
 
 
-def time_oracle(name, rows, min_seconds=0.0, reps=1):
+def time_oracle(name, rows, min_seconds=0.0, reps=1, nthreads=0):
     oracle, packed, s, ab, x, rows, K, B, G = oracle_sample(name, rows)
     wbytes = packed_bytes(rows, K, B, G)
     n = 0
     t0 = time.perf_counter()
     while True:
-        oracle.gemm(x, packed, s, ab, rows, K, B, G)
+        oracle.gemm(x, packed, s, ab, rows, K, B, G, nthreads=nthreads)
         n += 1
         el = time.perf_counter() - t0
         if n >= reps and el >= min_seconds:
@@ -464,6 +566,81 @@ def cpu_baseline(name):
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"the full {N}x{K} W{B} G{G} matrix at M={M}, {n} pass(es), "
                       f"{el:.1f} s, FP64 plain C over {cores} threads"}
+
+
+def _oracle_expert(tag, e, B, H, I, G, device):
+    """One expert's matrices from the seeded generator (drawn on the GPU, the
+    same values as on the CPU), packed by the oracle on the host."""
+    import oracle
+    import synthetic
+    u16 = lambda t: t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    gu = [t.cpu() for t in synthetic.matrix((tag, "gu", e), 2 * I, H, B, G, device=device)]
+    dn = [t.cpu() for t in synthetic.matrix((tag, "dn", e), H, I, B, G, device=device)]
+    return dict(B_gu=B, packed_gu=oracle.pack(gu[0].numpy(), B), scales_gu=gu[1].numpy(),
+                ab_gu=u16(gu[2]), B_dn=B, packed_dn=oracle.pack(dn[0].numpy(), B),
+                scales_dn=dn[1].numpy(), ab_dn=u16(dn[2]))
+
+
+def cpu_baselines(device):
+    """The oracle (FP64, plain C, all host threads unless stated) on bounded
+    samples of the other configurations, with what each sample was.  Timed:
+    the oracle's products only (input generation and packing excluded)."""
+    import oracle
+    import synthetic
+    out = []
+    cores = oracle.num_threads()
+    # config 1: the fitted W4 G128 256 x 1024 matrix at M = 1, in full
+    d = np.load(os.path.join(ROOT, "tests", "golden", "config1_w4g128.npz"))
+    x1 = synthetic.activations(1, 1, 1024).view(torch.int16).numpy().view(np.uint16)
+    n, t0 = 0, time.perf_counter()
+    while n < 3 or time.perf_counter() - t0 < 2.0:
+        oracle.gemm(x1, d["packed"], d["scales"], d["ab"], 256, 1024, 4, 128)
+        n += 1
+    el = time.perf_counter() - t0
+    out.append({"config": "W4 G128 256x1024 fitted (config 1), M=1", "value":
+                round(packed_bytes(256, 1024, 4, 128) * n / el / 1e9, 4), "unit": "GB/s",
+                "cores": cores, "sample": f"the full matrix, {n} passes, {el:.1f} s"})
+    # config 3: gate+up W2 at M = 1, 1024 of 6144 rows
+    gbs, el, n, _ = time_oracle("gate_up_m1", 1024, min_seconds=2.0)
+    out.append({"config": WORKLOADS["gate_up_m1"][0], "value": round(gbs, 4), "unit": "GB/s",
+                "cores": cores, "sample": f"1024 of 6144 rows, {n} passes, {el:.1f} s"})
+    # config 2 on one core
+    gbs, el, n, _ = time_oracle("down_m1", 512, min_seconds=2.0, nthreads=1)
+    out.append({"config": WORKLOADS["down_m1"][0], "value": round(gbs, 4), "unit": "GB/s",
+                "cores": 1, "sample": f"512 of 7168 rows on one thread, {n} passes, {el:.1f} s"})
+    # configs 4 and 5: whole routed-expert chains of sampled experts, scaled by
+    # the layer's active experts (the per-expert cost is the decode of its two
+    # matrices plus its routes' products)
+    H, I, E, k, G = 7168, 3072, 896, 16, 512
+    for cfg, T, routing, widths in [("config 4", 64, "uniform", "mixed"),
+                                    ("config 5", 8192, "zipf", "w4")]:
+        Bs = synthetic.expert_bits(4, E) if widths == "mixed" else torch.full((E,), 4)
+        if routing == "uniform":
+            ids, _ = synthetic.routing_uniform(4, T, E, k)
+        else:
+            ids, _ = synthetic.routing_zipf(5, T, E, k)
+        ids_np = ids.numpy()
+        x = synthetic.activations(7, T, H).view(torch.int16).numpy().view(np.uint16)
+        counts = np.bincount(ids_np.ravel(), minlength=E)
+        active = np.nonzero(counts)[0]
+        sample = [int(active[0]), int(active[len(active) // 2])]
+        spent, routes_done, expert_routes = 0.0, 0, 0
+        for e in sample:
+            ex = _oracle_expert(("cpu", cfg), e, int(Bs[e]), H, I, G, device)
+            rs = [int(r) for r in np.nonzero(ids_np.ravel() == e)[0]]
+            t0 = time.perf_counter()
+            oracle.moe_routes(x, ids_np, {e: ex}, H, I, G, routes=rs)
+            spent += time.perf_counter() - t0
+            routes_done += len(rs)
+        per_expert = spent / len(sample)
+        layer_s = per_expert * len(active)
+        out.append({"config": f"{cfg}: {T} tokens, top-16 over 896 experts ({widths})",
+                    "value": round(T / layer_s, 3), "unit": "tokens/s", "cores": cores,
+                    "sample": f"{len(sample)} experts ({routes_done} routes) timed in full, "
+                              f"{spent:.1f} s; layer time extrapolated to the "
+                              f"{len(active)} active experts ({layer_s:.0f} s)",
+                    "extrapolated": True})
+    return out
 
 
 def run_reference(args, world, rank):
@@ -525,27 +702,16 @@ def main():
     hbm, tf_burst, tf_sust, peak_src = load_peaks()
 
     main_res = time_gemm(cq, args.workload, args.steps, args.warmup, world, device,
-                         sample_clocks=True)
+                         sample_clocks=True, repeats=20)
     secondary = []
     if not args.no_secondary:
-        for name in ["gate_up_m1", "down_m16", "gate_up_m4096", "down_m4096"]:
+        for name in SECONDARY:
             if name == args.workload:
                 continue
             steps = 400 if WORKLOADS[name][5] <= 64 else 20
-            r = time_gemm(cq, name, steps, 3, world, device)
-            bound = "hbm" if r["M"] <= 64 else "tensor"
-            ent = {"workload": r["desc"], "ms_per_step": round(r["ms_per_step"], 5),
-                   "packed_gbs": round(r["gbs"] * world, 1),
-                   "tflops": round(r["tflops"] * world, 2)}
-            if bound == "hbm":
-                ach = r["alg_bytes"] / (r["ms_per_step"] * 1e-3) / 1e9
-                ent["roofline"] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
-                                   "unit": "GB/s", "frac": round(ach / hbm, 4)}
-            else:
-                ent["roofline"] = {"bound": "tensor", "achieved": round(r["tflops"], 1),
-                                   "peak": tf_burst, "unit": "TFLOP/s",
-                                   "frac": round(r["tflops"] / tf_burst, 4)}
-            secondary.append(ent)
+            r = time_gemm(cq, name, steps, 3, world, device, repeats=20)
+            secondary.append(gemm_entry(r, hbm, tf_burst, world))
+            torch.cuda.empty_cache()
 
     if not args.no_secondary and not args.no_moe:
         for name in ["moe_decode", "moe_prefill"]:
@@ -559,15 +725,18 @@ def main():
                    "mean_payload_bits_active": round(r["mean_payload_bits"], 4)}
             if name == "moe_decode":
                 ent["roofline"] = {"bound": "hbm", "achieved": round(r["gbs"], 1), "peak": hbm,
-                                   "unit": "GB/s", "frac": round(r["gbs"] / hbm, 4)}
+                                   "unit": "GB/s", "frac": round(r["gbs"] / hbm, 4),
+                                   "frac_nominal": round(r["gbs"] / NOMINAL_HBM_GBS, 4)}
             else:
                 ent["roofline"] = {"bound": "tensor", "achieved": round(r["tflops"], 1),
                                    "peak": tf_sust, "unit": "TFLOP/s",
                                    "frac": round(r["tflops"] / tf_sust, 4),
+                                   "frac_nominal": round(r["tflops"] / NOMINAL_BF16_TFLOPS, 4),
                                    "peak_kind": "sustained"}
             secondary.append(ent)
             torch.cuda.empty_cache()
 
+    cold = time_cold(cq, args.workload, device)
     e2e = time_e2e(cq, args.workload, args.steps, device)
     e2e["value"] = round(e2e["value"] * world, 3)
 
@@ -603,10 +772,18 @@ def main():
         "e2e": e2e,
         "gpu_launches": args.steps,
         "clocks": r["clocks"],
+        "timing": {"method": "one replay of a CUDA graph of the K steps, CUDA events on the "
+                             "launching stream, a spin kernel queued ahead of the first event",
+                   "repeats": len(r.get("rep_ms_per_step", [])),
+                   "best_ms_per_step": round(min(r["rep_ms_per_step"]), 6),
+                   "median_ms_per_step": round(statistics.median(r["rep_ms_per_step"]), 6),
+                   "cold_launch": cold},
+        "frac_nominal_hbm": round(ach / NOMINAL_HBM_GBS, 4),
         "secondary": secondary,
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload)
+        line["cpu_baselines"] = cpu_baselines(device)
     print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

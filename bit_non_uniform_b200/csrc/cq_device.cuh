@@ -151,6 +151,12 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 
+// Prefetch [src, src + bytes) into L2 (bulk, asynchronous, nothing tracked).
+// src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // 32-bit global load through the read-only path whose place in the
 // instruction stream is kept (volatile): issued before the loads after it.
 __device__ __forceinline__ uint32_t ldg_u32_ordered(const void* ptr) {

@@ -60,10 +60,18 @@ static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int B, int epilogue, 
 // tensor-core engine.  (The test hook may force one of them.)
 enum GemmPath { PATH_AUTO = 0, PATH_NARROW = 1, PATH_GEMV = 2, PATH_ENGINE = 3 };
 
+// The narrow-row kernel takes 3 <= M <= 5 on its own: the GEMV is faster for
+// M <= 2 and the engine from about M = 6 (down_proj 7168 x 3072 W3 and
+// gate_up 6144 x 7168 W2, graphs of launches over weights larger than L2).
+constexpr int64_t kNrAutoMinM = 3, kNrAutoMaxM = 5;
+static bool narrow_wanted(int64_t M, int path) {
+  return path == PATH_NARROW || (path == PATH_AUTO && M >= kNrAutoMinM && M <= kNrAutoMaxM);
+}
+
 // Scratch bytes of whichever path gemm_impl takes for this problem.
 static void gemm_scratch(int64_t M, int64_t N, int64_t K, int B, int G, int epilogue, int sms,
                          size_t* counter_bytes, size_t* total, int path = PATH_AUTO) {
-  if (path == PATH_AUTO || path == PATH_NARROW) {
+  if (narrow_wanted(M, path)) {
     const NrPlan nv = plan_narrow(M, N, K, B, G, epilogue, sms);
     if (nv.use) {
       *counter_bytes = nv.ws_counter_bytes;
@@ -151,7 +159,7 @@ int gemm_impl(const uint16_t* x, int64_t M, const uint8_t* packed, const float* 
   const int sms = num_sms();
   if (sms <= 0) return CQ_ERR_CUDA;
   if (debug_skip) path = PATH_ENGINE;
-  if (path == PATH_AUTO || path == PATH_NARROW) {
+  if (narrow_wanted(M, path)) {
     const NrPlan nv = plan_narrow(M, N, K, B, G, epilogue, sms);
     if (nv.use) {
       const size_t need = nv.ws_counter_bytes + nv.ws_partial_bytes;

@@ -26,27 +26,30 @@
 // hold the gate and up value of the same output).  A unit is (row block rb,
 // slice step j): the 16 rows times slice j of each quarter, 8192 weights.
 // Units are numbered rb-major and split evenly over the CTAs (one per SM).  A
-// CTA builds the level tables of every (row, group) its units touch while its
-// first loads are in flight; its warps then take the units round robin, row
-// block by row block when every slice step's activations fit in shared
-// memory (else slice step by slice step, through a ring of activation
-// stages).  A unit's partial sums go to a shared-memory slot; the warp that
-// finishes a row block's last unit sums the row block's slots (slice steps
-// in order) and writes it out.  A row block shared by consecutive CTAs is
-// finished early by the later ones (it is the first row block they do),
-// which park their parts in the workspace; the first CTA (the owner, which
-// does it last) adds them in CTA order.  Results are run-to-run
-// deterministic.
+// CTA builds the level tables of every (row, group) its units touch; its
+// warps then take the units round robin and leave each unit's partial sums
+// in a shared-memory slot.  After one barrier, warp r sums the slots of the
+// CTA's row block r (slice steps in order) and writes it out.  A row block
+// shared by consecutive CTAs: the later CTAs park their parts in the
+// workspace and count them; the first CTA (the owner) waits for the count
+// and adds the parts in CTA order.  A CTA publishes its own part before it
+// waits for any, so the waits form a chain that ends at the last CTA.
+// Results are run-to-run deterministic.
 //
 // Loads.  Each warp loads the codes of its own units straight into registers
 // with 16-byte global loads (the lane's two rows of one slice of its
-// quarter), ahead of its decoding, and the CTA stages its activations once,
-// with 16-byte asynchronous copies, as [slice step][k pair][token][quarter]
-// [8 values], so that a warp's 16-byte activation loads are conflict free.
-// (Box copies of 16 rows x 4 quarters x one 48-byte slice came in too
-// slowly: the copy engine handles such short rows at a few bytes per
-// cycle.)  No shared-memory ring, no producer warp: eight warps build the
-// tables, decode, multiply and finish row blocks.
+// quarter), NB units ahead of its decoding, and the CTA stages its
+// activations once, with 16-byte asynchronous copies, as [slice step][k pair]
+// [token][quarter][8 values], so that a warp's 16-byte activation loads are
+// conflict free.  No fence or barrier lies between a warp's first code load
+// and its last unit: a fence (and a barrier, which orders memory like one)
+// waits until the loads in flight have landed, which would stop the warp
+// until the codes of its later units arrive.  The CTA's rows are also
+// prefetched into L2 in a few bulk requests at the start.  (Box copies of 16
+// rows x 4 quarters x one 48-byte slice came in too slowly: the copy engine
+// handles such short rows at a few bytes per cycle.)  No shared-memory ring,
+// no producer warp: eight warps build the tables, decode, multiply and
+// finish row blocks.
 //
 // This is the narrow-row GEMV of the article's A16 path ("压缩权重必须“边解码、
 // 边计算”"): codes and group parameters -> levels generated in the tile ->
@@ -64,11 +67,12 @@ namespace cq {
 constexpr int kNrCompute = 8;                   // warps
 constexpr int kNrThreads = kNrCompute * 32;
 constexpr int kNrMaxRbl = 8;                    // row blocks one CTA may touch
+static_assert(kNrMaxRbl <= kNrCompute, "one warp sums each row block");
 constexpr int kNrMaxUnits = 96;                 // units one CTA may own
 constexpr int kNrMaxJ = 64;                     // slice steps per quarter (K <= 32768)
 constexpr int kNrPreItems = 4;                  // table items per thread loaded up front
-// flags, and per row block the units of the CTA and how many of them are done
-constexpr int kNrBarBytes = 64 + 8 * kNrMaxRbl;
+// flags
+constexpr int kNrBarBytes = 64;
 // the processing order of a CTA's units and its inverse (unit of (rbl, j))
 constexpr int kNrOrderBytes = 4 * (kNrMaxUnits + kNrMaxRbl * kNrMaxJ);
 
@@ -216,10 +220,14 @@ __device__ __noinline__ bool nr_finish_row_block(const NarrowParams& p, int cta,
     float* dst = p.partial + (static_cast<int64_t>(cta) * 32 + lane) * NV;
 #pragma unroll
     for (int k = 0; k < NV; ++k) __stcg(dst + k, v[k]);
+    const long long t_f = p.trace ? clock64() : 0;
     __threadfence();
     __syncwarp();
     if (lane == 0) atomicAdd(p.counter + rb, 1);
-    if (lane == 0 && p.trace) p.trace[blockIdx.x * 64 + 40] = clock64();
+    if (lane == 0 && p.trace) {
+      p.trace[blockIdx.x * 64 + 40] = clock64();
+      p.trace[blockIdx.x * 64 + 43] = clock64() - t_f;
+    }
     return true;
   }
   if (lane == 0 && p.trace) p.trace[blockIdx.x * 64 + 41] = clock64();
@@ -300,8 +308,6 @@ __global__ void __launch_bounds__(kNrThreads, 1)
   const uint32_t xs0 = base + p.x_off;
   const uint32_t fl = raw + static_cast<uint32_t>(p.smem_bytes - kNrBarBytes - kNrOrderBytes);
   volatile int* const flags = reinterpret_cast<volatile int*>(smem_raw + (fl - raw));
-  int* const cnt_rb = const_cast<int*>(flags + 16);         // [rbl] the CTA's units of it
-  int* const done_rb = cnt_rb + kNrMaxRbl;                  // [rbl] of those, finished
   // order[i] of the CTA's units in processing order: rbl | j << 8;
   // inv[rbl * kNrMaxJ + j] = i
   int* const order = reinterpret_cast<int*>(smem_raw + (fl + kNrBarBytes - raw));
@@ -327,18 +333,14 @@ __global__ void __launch_bounds__(kNrThreads, 1)
     if (n_units < 1 || n_units > p.max_units || n_units > kNrMaxUnits || n_rbl > p.max_rbl ||
         n_rbl > kNrMaxRbl || p.Q > kNrMaxJ || p.M < 1 || p.M > MT)
       bad = 40;
-    // processing order: row block by row block (a row block shared with the
-    // previous CTA comes first and is finished early)
+    // processing order: row block by row block
     int i = 0;
     for (int rbl = 0; rbl < n_rbl && !bad; ++rbl) {
-      cnt_rb[rbl] = 0;
-      done_rb[rbl] = 0;
       for (int j = 0; j < p.Q; ++j) {
         const int u = (rb_lo + rbl) * p.Q + j;
         if (u >= u0 && u < u1) {
           inv[rbl * kNrMaxJ + j] = i;
           order[i++] = rbl | (j << 8);
-          ++cnt_rb[rbl];
         }
       }
     }
@@ -353,6 +355,29 @@ __global__ void __launch_bounds__(kNrThreads, 1)
   griddep_wait();
   if (tid == 0) NR_STAMP(4);
   if (flags[0]) return;
+  // the rows of this CTA's row blocks, brought into L2 in a few bulk
+  // prefetches: the lanes' 16-byte code loads then hit L2
+  if (warp == 0 && lane < n_rbl * 2) {
+    const int rb = rb_lo + (lane >> 1), half = lane & 1;
+    if (rb < p.n_rb) {
+      int r0, nrows;
+      if (p.epilogue == CQ_EPI_SWIGLU) {
+        r0 = (half ? (p.N >> 1) : 0) + rb * 8;
+        nrows = 8;
+      } else {
+        r0 = rb * 16 + half * 8;
+        nrows = min(8, p.N - r0);
+      }
+      if (nrows > 0) {
+        const int64_t bytes = static_cast<int64_t>(nrows) * p.row_bytes;
+        const uint8_t* src = p.packed + static_cast<int64_t>(r0) * p.row_bytes;
+        for (int64_t o = 0; o < bytes; o += (1 << 20)) {
+          const int64_t n = bytes - o < (1 << 20) ? bytes - o : (1 << 20);
+          prefetch_l2_bulk(src + o, static_cast<uint32_t>(n));
+        }
+      }
+    }
+  }
 
   // -------------------------------------------------------- level tables
   // block (rbl, it, lgi) holds the tables of lanes (g, c) = rows (rb, it, g)
@@ -375,7 +400,7 @@ __global__ void __launch_bounds__(kNrThreads, 1)
       }
     }
 
-  // -------------------------------------------- loads: activations, codes
+  // ------------------------------------------------------- activations
   // every slice step's activations, as 16-byte chunks (j, s'', m, c)
   {
     const int n_chunks = p.Q * 16 * p.M * 4;
@@ -390,19 +415,6 @@ __global__ void __launch_bounds__(kNrThreads, 1)
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   }
-  // codes of this warp's first units (registers)
-  uint32_t cn0[NB][4 * B], cn1[NB][4 * B];
-#pragma unroll
-  for (int k = 0; k < NB; ++k) {
-    const int i = warp + k * kNrCompute;
-#pragma unroll
-    for (int w = 0; w < 4 * B; ++w) cn0[k][w] = cn1[k][w] = 0u;
-    if (i < n_units) {
-      const int ord = order[i];
-      nr_load_codes<B>(p, rb_lo + (ord & 255), ord >> 8, g, c, cn0[k], cn1[k]);
-    }
-  }
-
   {
     for (int k = 0, id = tid; id < n_items; ++k, id += kNrThreads) {
       const int ln = id & 31;
@@ -439,11 +451,26 @@ __global__ void __launch_bounds__(kNrThreads, 1)
   cp_async_wait_all();
   __syncthreads();
   if (tid == 0) NR_STAMP(2);
+  // codes of this warp's first units (registers).  From here to the end of
+  // the units no fence or barrier is passed: either would wait for these
+  // loads, and for the ones issued NB units ahead inside the loop.
+  uint32_t cn0[NB][4 * B], cn1[NB][4 * B];
+#pragma unroll
+  for (int k = 0; k < NB; ++k) {
+    const int i = warp + k * kNrCompute;
+#pragma unroll
+    for (int w = 0; w < 4 * B; ++w) cn0[k][w] = cn1[k][w] = 0u;
+    if (i < n_units) {
+      const int ord = order[i];
+      nr_load_codes<B>(p, rb_lo + (ord & 255), ord >> 8, g, c, cn0[k], cn1[k]);
+    }
+  }
+
 
   // ------------------------------------------------------------ the units
-  long long cyc_work = 0, cyc_fin = 0;
-  bool ok = true;
-  for (int i = warp; i < n_units && ok; i += kNrCompute) {
+  long long cyc_work = 0;
+  if (p.trace && lane == 0) p.trace[blockIdx.x * 64 + 44 + warp] = clock64();
+  for (int i = warp; i < n_units; i += kNrCompute) {
     const long long t_a = p.trace ? clock64() : 0;
     const int ord = order[i];
     const int rbl = ord & 255, j = ord >> 8;
@@ -532,28 +559,21 @@ __global__ void __launch_bounds__(kNrThreads, 1)
     for (int h = 0; h < MT / 8; ++h)
 #pragma unroll
       for (int b = 0; b < 4; ++b) sl[h * 4 + b] = acc[0][h][b] + acc[1][h][b];
-    // the warp that finishes a row block's last unit in this CTA sums it
-    __threadfence_block();
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) last = atomicAdd(done_rb + rbl, 1) + 1 == cnt_rb[rbl];
-    last = __shfl_sync(0xffffffffu, last, 0);
-    const long long t_c = p.trace ? clock64() : 0;
-    if (last) {
-      __threadfence_block();
-      if (!nr_finish_row_block<MT>(p, cta, rb_lo + rbl, u0, u1, rbl, inv, slot_f, lane,
-                                   flags + 2))
-        ok = false;
-    }
-    if (p.trace) {
-      cyc_work += t_c - t_a;
-      cyc_fin += clock64() - t_c;
-    }
+    if (p.trace) cyc_work += clock64() - t_a;
   }
+  // ------------------------------------------------------- the row blocks
+  // every unit is in its slot; warp rbl sums row block rbl (a row block
+  // shared with the next CTA waits for that CTA's part, which it publishes
+  // here too, after its own units: no CTA waits before publishing)
+  __syncthreads();
+  const long long t_c = p.trace ? clock64() : 0;
+  if (warp < n_rbl)   // a wait that gives up sets the error flag itself
+    nr_finish_row_block<MT>(p, cta, rb_lo + warp, u0, u1, warp, inv, slot_f, lane, flags + 2);
   if (p.trace && lane == 0) {
+    p.trace[blockIdx.x * 64 + 52 + warp] = t_c;
     p.trace[blockIdx.x * 64 + 8 + 3 * warp] = 0;
     p.trace[blockIdx.x * 64 + 9 + 3 * warp] = cyc_work;
-    p.trace[blockIdx.x * 64 + 10 + 3 * warp] = cyc_fin;
+    p.trace[blockIdx.x * 64 + 10 + 3 * warp] = clock64() - t_c;
   }
   __syncthreads();
   if (tid == 0) NR_STAMP(1);

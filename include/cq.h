@@ -119,11 +119,12 @@ CQ_API int cq_decode(const uint8_t *packed, const float *scales, const uint16_t 
  *              counters that must be zero before the first call that uses
  *              the buffer; every completed call leaves them zero again.
  * Calls that share one workspace must not overlap on the GPU.
- * Paths: M <= 16 with K a multiple of 512 runs the narrow-row kernel
+ * Paths: M <= 2 runs the decode-sized GEMV kernel (no workspace) where its
+ * plan fits; 3 <= M <= 5 with K a multiple of 512 runs the narrow-row kernel
  * ([CQ] "压缩权重必须“边解码、边计算”": the narrow-row GEMV; register-operand
  * tensor-core MMAs, 16-row x one-slice work units split evenly over the SMs,
- * row blocks shared by two CTAs summed through the workspace); other M <= 2
- * shapes run the decode-sized GEMV kernel (no workspace); everything else
+ * row blocks shared by two CTAs summed through the workspace), also the
+ * fallback of M <= 2 shapes the GEMV does not take; everything else
  * runs the tensor-core engine (128-row weight tiles, 16- to 192-token
  * activation tiles, stream-K over the K slices, partial tiles summed in a
  * fixed order).  Results are run-to-run deterministic.  All three kernels
