@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int64_t x = r0; ok && x < r1 && !*abort_flag;) {
         const Segment sg = segment_at(x, r1, p.spt);
-        const TileInfo ti = resolve_tile(p, sg.t, NT);
+        const TileInfo ti = resolve_tile(p, sg.t, NT, 2, 4);
         const int Bw = ti.mat.B;
         const int row_a = tile_row(p, ti.rt, 0);
         const int row_b = tile_row(p, ti.rt, 64);
@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int64_t x = r0; ok && x < r1;) {
       const Segment sg = segment_at(x, r1, p.spt);
-      const TileInfo ti = resolve_tile(p, sg.t, NT);
+      const TileInfo ti = resolve_tile(p, sg.t, NT, 2, 4);
       const int Bw = ti.mat.B;
       const int grow = tile_row(p, ti.rt, i);
       const uint32_t swz = Bw == 2 ? ((i >> 2) & 1u) : (Bw == 4 ? ((i >> 1) & 3u) : 0u);
@@ -549,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int64_t x = r0; ok && x < r1;) {
       const Segment sg = segment_at(x, r1, p.spt);
-      const TileInfo ti = resolve_tile(p, sg.t, NT);
+      const TileInfo ti = resolve_tile(p, sg.t, NT, 2, 4);
       const int grow = tile_row(p, ti.rt, i);
       const int nchunks = (ti.m_valid + 15) >> 4;
       const int g0 = sg.s0 / spc, g1 = (sg.s1 - 1) / spc;

@@ -61,7 +61,9 @@ constexpr int kMmaWarp = 9;
 constexpr int kEpiWarp0 = 10;
 
 // NT: token-tile width; TE: entries of a row's pair table (16 when every
-// matrix of the launch has B = 2 or 4, 64 when one may have B = 3).
+// matrix of the launch has B = 2 or 4, 64 when one may have B = 3), or 0 for
+// the wide-code decoder (any B in 1..8, levels evaluated per code, no
+// tables, slices of up to 128 bytes per row).
 template <int NT, int TE>
 struct EngineCfg {
   static constexpr int SPS = NT <= 32 ? 4 : (NT == 64 ? 2 : 1);   // slices per stage
@@ -73,7 +75,9 @@ struct EngineCfg {
   static constexpr int NBUF = FREE2 >= 2 ? 2 : 1;
   static constexpr int RING = FREE2 >= 4 ? 4 : (FREE2 >= 2 ? FREE2 : kTmemRing);
   static constexpr int DCOL = RING * 64;                        // first accumulator column
-  static constexpr int SLICE_W_BYTES = kRows * 16 * 4;          // one slice of packed rows (B<=4)
+  static constexpr int BMIN = TE == 0 ? 1 : 2;                  // code widths of the launch
+  static constexpr int BMAX = TE == 0 ? 8 : 4;
+  static constexpr int SLICE_W_BYTES = kRows * 16 * BMAX;       // one slice of packed rows
   static constexpr int W_STAGE = SPS * SLICE_W_BYTES;           // codes of SPS slices
   static constexpr int X_STAGE = 256 * SPS * NT;                // 2*SPS boxes of 64 x NT bf16
   static constexpr int XCHG_BYTES = 16 * 64 * 4;
@@ -192,7 +196,8 @@ struct TileInfo {
 // Tile t of the launch.  Plain mode: t = tt * n_rt + rt.  Grouped mode:
 // experts in order, each contributing n_rt x ntt(e) tiles (tt fastest), so
 // expert e owns tiles [n_rt * ttpre[e], n_rt * ttpre[e+1]).
-__device__ __forceinline__ TileInfo resolve_tile(const EngineParams& p, int t, int NT) {
+__device__ __forceinline__ TileInfo resolve_tile(const EngineParams& p, int t, int NT,
+                                                 int bmin, int bmax) {
   TileInfo ti;
   if (!p.grouped) {
     ti.mat = p.mat;
@@ -220,6 +225,12 @@ __device__ __forceinline__ TileInfo resolve_tile(const EngineParams& p, int t, i
   ti.tt = local - ti.rt * ntt;
   const LayerEntry* le = p.layer + e;
   ti.mat = le->mat[p.which];
+  if (ti.mat.B < bmin || ti.mat.B > bmax) {
+    // a width this launch's rings and tables were not sized for: flag it and
+    // decode a width that stays inside them
+    bad_access(28);
+    ti.mat.B = 2;
+  }
   ti.wmap = &le->map[p.which];
   ti.x_row0 = ld_guarded(p.g_off + e) + ti.tt * NT;
   const int rem = ld_guarded(p.g_cnt + e) - ti.tt * NT;
@@ -391,6 +402,95 @@ __device__ __forceinline__ void decode_half_slice_to_tmem(const uint4* codes, ui
   uint32_t r[32];
   decode_half<B, 32 * HALF>(c, tbl, i, r);
   tmem_st32(taddr, r);
+}
+
+// Wide-code decoder (TE = 0): the level of every code is evaluated on the
+// spot, with the same FP64 steps as a table entry (q(t) in FP64, times s,
+// rounded once to FP32 and then to BF16).  A 2^B-entry table per row would
+// not fit beside the rings for B = 8, and for G = 512 building it costs
+// about as much as evaluating each code once.  t = |k| / Kc is taken as
+// |k| * (1 / Kc): exact for |k| in {0, Kc}, elsewhere within one FP64 ulp of
+// the quotient, 2^-45 of a BF16 step.
+struct WideRow {
+  double a, b, c, rinv;   // shape parameters, c = 1 - a - b, 1 / Kc'
+  float s;                // group scale (0 for rows past N)
+  int mult, off;          // k' = mult * u - off: midrise 2u - (2^B - 1), midtread u - Kc
+};
+
+__device__ __forceinline__ WideRow wide_row(bool valid, float s, uint32_t abw, int mode, int B) {
+  WideRow w;
+  w.a = static_cast<double>(__half2float(__ushort_as_half(abw & 0xFFFFu)));
+  w.b = static_cast<double>(__half2float(__ushort_as_half(abw >> 16)));
+  w.c = 1.0 - w.a - w.b;
+  w.s = valid ? s : 0.f;
+  w.mult = mode == CQ_GRID_MIDRISE ? 2 : 1;
+  w.off = mode == CQ_GRID_MIDRISE ? (1 << B) - 1 : (1 << (B - 1)) - 1;
+  w.rinv = 1.0 / static_cast<double>(w.off > 0 ? w.off : 1);
+  return w;
+}
+
+// FP32 level of code u before the sign (|s q(t)|), and whether k < 0.
+__device__ __forceinline__ float wide_level(const WideRow& w, uint32_t u, bool& neg) {
+  const int k = w.mult * static_cast<int>(u) - w.off;
+  neg = k < 0;
+  const int ak = k < 0 ? -k : k;
+  // |k| as a double without a conversion instruction: 2^52 + ak, minus 2^52
+  double t = (__hiloint2double(0x43300000, ak) - 4503599627370496.0) * w.rinv;
+  if (ak == w.off) t = 1.0;
+  const double q = t * (w.a + t * (w.b + t * w.c));
+  return static_cast<float>(static_cast<double>(w.s) * q);
+}
+
+// The B-bit code at bit offset o of the slice words c[] (LSB first).
+template <int B>
+__device__ __forceinline__ uint32_t code_at(const uint32_t (&c)[4 * B], int o) {
+  const int wi = o >> 5, sh = o & 31;
+  uint32_t v;
+  if (sh + B <= 32)
+    v = c[wi] >> sh;
+  else
+    v = __funnelshift_r(c[wi], c[wi + 1 < 4 * B ? wi + 1 : 4 * B - 1], sh);
+  return v & ((1u << B) - 1u);
+}
+
+// Decode pairs [32*HALF, 32*HALF+32) of one slice of a B-bit row into TMEM
+// columns taddr .. taddr+31: the wide-code counterpart of
+// decode_half_slice_to_tmem.
+template <int B, int HALF>
+__device__ __forceinline__ void decode_wide_half_to_tmem(const uint4* codes, uint32_t swz,
+                                                         const WideRow& w, uint32_t taddr) {
+  uint32_t c[4 * B];
+#pragma unroll
+  for (int v = 0; v < B; ++v) {
+    if ((v + 1) * 128 > HALF * 32 * 2 * B && v * 128 < (HALF + 1) * 32 * 2 * B) {
+      const uint4 q = codes[v ^ swz];
+      c[4 * v + 0] = q.x;
+      c[4 * v + 1] = q.y;
+      c[4 * v + 2] = q.z;
+      c[4 * v + 3] = q.w;
+    } else {
+      c[4 * v + 0] = c[4 * v + 1] = c[4 * v + 2] = c[4 * v + 3] = 0u;
+    }
+  }
+  uint32_t r[32];
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const int pr = 32 * HALF + q;                 // pair: codes 2pr (low) and 2pr+1 (high)
+    bool n0, n1;
+    const float l0 = wide_level(w, code_at<B>(c, 2 * pr * B), n0);
+    const float l1 = wide_level(w, code_at<B>(c, (2 * pr + 1) * B), n1);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(l0, l1);
+    r[q] = *reinterpret_cast<const uint32_t*>(&h) ^ (n0 ? 0x8000u : 0u) ^
+           (n1 ? 0x80000000u : 0u);
+  }
+  tmem_st32(taddr, r);
+}
+
+template <int B>
+__device__ __forceinline__ void decode_wide_slice_to_tmem(const uint4* codes, uint32_t swz,
+                                                          const WideRow& w, uint32_t taddr) {
+  decode_wide_half_to_tmem<B, 0>(codes, swz, w, taddr);
+  decode_wide_half_to_tmem<B, 1>(codes, swz, w, taddr + 32);
 }
 
 // ---------------------------------------------------------------------------
@@ -627,7 +727,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int64_t x = r0; ok && x < r1 && !*abort_flag;) {
         const Segment sg = segment_at(x, r1, p.spt);
-        const TileInfo ti = resolve_tile(p, sg.t, NT);
+        const TileInfo ti = resolve_tile(p, sg.t, NT, C::BMIN, C::BMAX);
         const int Bw = ti.mat.B;
         // first weight row of the two 64-row boxes of this tile
         const int row_a = tile_row(p, ti.rt, 0);
@@ -792,16 +892,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int spc = p.G / kSlice;                        // slices per group
     for (int64_t x = r0; ok && x < r1;) {
       const Segment sg = segment_at(x, r1, p.spt);
-      const TileInfo ti = resolve_tile(p, sg.t, NT);
+      const TileInfo ti = resolve_tile(p, sg.t, NT, C::BMIN, C::BMAX);
       const int Bw = ti.mat.B;
       const int grow = tile_row(p, ti.rt, i);
       // 16-byte chunk v of this row sits at chunk (v ^ swz) of the row (TMA swizzle)
-      const uint32_t swz = Bw == 2 ? ((i >> 2) & 1u) : (Bw == 4 ? ((i >> 1) & 3u) : 0u);
+      const uint32_t swz =
+          Bw == 2 ? ((i >> 2) & 1u) : (Bw == 4 ? ((i >> 1) & 3u) : (Bw == 8 ? (i & 7u) : 0u));
       const bool valid = grow < p.N;
       // group metadata: the current group and a prefetch of the next group
       // this thread meets (its first slice of this segment, then after each
       // switch the group of its first slice past the current group)
       int cur_g = -1;
+      WideRow wr = {};
       const int s_first = sg.s0 + ((sg.s0 & 1) != h ? 1 : 0);
       float s_next = 0.f;
       uint32_t ab_next = 0;
@@ -827,7 +929,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int sl = sb + j;
           if ((sl & 1) == h) {
             const int g = sl / spc;
-            if (TE < 64 && Bw == 3) {
+            if (TE == 16 && Bw == 3) {
               // a 64-entry table does not fit this launch's tables (the host
               // never plans it): record it and leave the table alone
               if (g != cur_g && i == 0) bad_access(27);
@@ -846,7 +948,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 s_next = __ldg(ti.mat.scales + static_cast<int64_t>(grow) * ng + gn);
                 ab_next = __ldg(ti.mat.ab + static_cast<int64_t>(grow) * ng + gn);
               }
-              if (Bw == 2)
+              if constexpr (TE == 0)
+                wr = wide_row(valid, s_cur, ab_cur, p.mode, Bw);
+              else if (Bw == 2)
                 build_table_all<2>(mytbl, i, valid, s_cur, ab_cur, p.mode);
               else if (Bw == 3)
                 build_table_all<3>(mytbl, i, valid, s_cur, ab_cur, p.mode);
@@ -865,7 +969,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t taddr = tmem_base + lane_off + ts * 64;
             const uint4* caddr =
                 reinterpret_cast<const uint4*>(gbase + (wrow + j * C::SLICE_W_BYTES - base));
-            if (Bw == 2) {
+            if constexpr (TE == 0) {
+              switch (Bw) {
+                case 1: decode_wide_slice_to_tmem<1>(caddr, swz, wr, taddr); break;
+                case 2: decode_wide_slice_to_tmem<2>(caddr, swz, wr, taddr); break;
+                case 3: decode_wide_slice_to_tmem<3>(caddr, swz, wr, taddr); break;
+                case 4: decode_wide_slice_to_tmem<4>(caddr, swz, wr, taddr); break;
+                case 5: decode_wide_slice_to_tmem<5>(caddr, swz, wr, taddr); break;
+                case 6: decode_wide_slice_to_tmem<6>(caddr, swz, wr, taddr); break;
+                case 7: decode_wide_slice_to_tmem<7>(caddr, swz, wr, taddr); break;
+                default: decode_wide_slice_to_tmem<8>(caddr, swz, wr, taddr); break;
+              }
+            } else if (Bw == 2) {
               decode_half_slice_to_tmem<2, 0>(caddr, swz, mytbl, i, taddr);
               decode_half_slice_to_tmem<2, 1>(caddr, swz, mytbl, i, taddr + 32);
             } else if (Bw == 3) {
@@ -907,7 +1022,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int64_t x = r0; ok && x < r1;) {
       const Segment sg = segment_at(x, r1, p.spt);
-      const TileInfo ti = resolve_tile(p, sg.t, NT);
+      const TileInfo ti = resolve_tile(p, sg.t, NT, C::BMIN, C::BMAX);
       const int grow = tile_row(p, ti.rt, i);
       const uint32_t db = C::NBUF == 2 ? (seg & 1u) : 0u;
       const uint32_t duse = C::NBUF == 2 ? (seg >> 1) : seg;

@@ -13,6 +13,10 @@ namespace cq {
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;   // 2 s per wait
 
+// The widths the engine decodes through pair tables; the others (1, 5..8)
+// take its wide-code decoder, with token tiles of at most 128.
+static bool table_width(int B) { return B >= 2 && B <= 4; }
+
 // Token-tile width.  Each token tile decodes the weights again, and up to
 // N = 192 the decode of a slice costs more than its MMAs, so wide problems
 // take wide tiles with two accumulator buffers in TMEM (beside a ring of two
@@ -25,7 +29,7 @@ static int pick_nt(int64_t M, int B) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
-  if (M <= 128) return 128;
+  if (M <= 128 || !table_width(B)) return 128;
   const int64_t pad128 = (M + 127) / 128 * 128;
   if (B == 3) {
     const int64_t pad176 = (M + 175) / 176 * 176;
@@ -118,10 +122,15 @@ static int launch_engine(const EngineParams& p, const CUtensorMap& map, const CU
 }
 
 // Pair tables of 64 entries for W3, 16 for W2/W4 (the smaller tables leave
-// room for more activation stages).
+// room for more activation stages); the wide-code decoder for the other
+// widths (token tiles of at most 128).
 template <int NT>
 static int launch_engine_te(const EngineParams& p, const CUtensorMap& map,
                             const CUtensorMap& wmap, int B, cudaStream_t s) {
+  if (!table_width(B)) {
+    if constexpr (NT <= 128) return launch_engine<NT, 0>(p, map, wmap, s);
+    return CQ_ERR_UNSUPPORTED;              // pick_nt never plans it
+  }
   if (B == 3) return launch_engine<NT, 64>(p, map, wmap, s);
   return launch_engine<NT, 16>(p, map, wmap, s);
 }
@@ -131,7 +140,7 @@ static int launch_engine_te(const EngineParams& p, const CUtensorMap& map,
 static int validate_gemm(const uint16_t* x, int64_t M, const uint8_t* packed,
                          const float* scales, const uint16_t* ab, int64_t N, int64_t K, int B,
                          int G, int grid_mode, int epilogue, int out_dtype, const void* y) {
-  int st = validate_matrix(packed, scales, ab, N, K, B, G, grid_mode);
+  int st = validate_matrix(packed, scales, ab, N, K, B, G, grid_mode, 1, 8);
   if (st != CQ_OK) return st;
   if (M < 0) return CQ_ERR_INVALID_ARG;
   if (epilogue != CQ_EPI_NONE && epilogue != CQ_EPI_SWIGLU) return CQ_ERR_INVALID_ARG;

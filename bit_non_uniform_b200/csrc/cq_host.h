@@ -34,8 +34,9 @@ inline bool ensure_smem_limit(Kernel* kernel, int bytes, std::atomic<uint64_t>& 
   return true;
 }
 
-// Bit widths: the GEMM paths take B in {2, 3, 4}; the format tools (pack,
-// decode) take 1..8 (the midtread grid needs B >= 2: Kc = 2^(B-1) - 1 > 0).
+// Bit widths: cq_gemm and the format tools (pack, decode) take 1..8 (the
+// midtread grid needs B >= 2: Kc = 2^(B-1) - 1 > 0); the grouped MoE GEMM and
+// the Dynamic A8 path take {2, 3, 4}.
 inline int validate_matrix(const uint8_t* packed, const float* scales, const uint16_t* ab,
                            int64_t N, int64_t K, int B, int G, int grid_mode, int b_min = 2,
                            int b_max = 4) {
@@ -92,8 +93,9 @@ inline int encode_bf16_rows_sw128(CUtensorMap* map, const void* base, int64_t ro
 
 // Tensor map over a packed CubicQuant matrix viewed as uint8 [rows][row_bytes],
 // loaded as boxes of 16*B bytes (one 128-code slice) x 64 rows.  The swizzle
-// (32-byte for B=2, 64-byte for B=4, none for B=3's 48-byte rows) keeps the
-// row-per-thread 16-byte shared-memory reads of the decoders conflict free.
+// (32-byte for B=2, 64-byte for B=4, 128-byte for B=8, none for the odd
+// widths' 16*B-byte rows and for B=6) keeps the row-per-thread 16-byte
+// shared-memory reads of the decoders conflict free (B=6: two-way).
 inline int encode_packed_rows(CUtensorMap* map, const void* base, int64_t rows,
                               int64_t row_bytes, int B) {
   EncodeTiledFn fn = encode_tiled_fn();
@@ -102,8 +104,10 @@ inline int encode_packed_rows(CUtensorMap* map, const void* base, int64_t rows,
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(16 * B), 64u};
   cuuint32_t estr[2] = {1u, 1u};
-  CUtensorMapSwizzle sw = B == 2 ? CU_TENSOR_MAP_SWIZZLE_32B
-                                 : (B == 4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE);
+  CUtensorMapSwizzle sw = B == 2   ? CU_TENSOR_MAP_SWIZZLE_32B
+                          : B == 4 ? CU_TENSOR_MAP_SWIZZLE_64B
+                          : B == 8 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                   : CU_TENSOR_MAP_SWIZZLE_NONE;
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

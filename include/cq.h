@@ -34,8 +34,10 @@
  *     NULL = legacy default stream) and returns a cq_status.  Arguments are
  *     validated on the host before anything is launched; on error nothing
  *     is launched and no output is touched.
- *   - Supported: B in {2,3,4} for cq_gemm, cq_gemm_noalloc and the MoE
- *     layer, B in 1..8 for cq_pack and cq_decode (midtread: 2..8);
+ *   - Supported: B in 1..8 for cq_pack, cq_decode, cq_gemm and
+ *     cq_gemm_noalloc (midtread: 2..8; the 8-bit code stream of [CQ]
+ *     "为什么只用两个形状参数？" is an ordinary 1..8-bit integer stream);
+ *     B in {2,3,4} for the MoE layer and the Dynamic A8 path;
  *     G a multiple of 128; K a multiple of G;
  *     N >= 1; packed / x / y / workspace 16-byte aligned; scales and ab
  *     4-byte aligned.
@@ -119,15 +121,20 @@ CQ_API int cq_decode(const uint8_t *packed, const float *scales, const uint16_t 
  *              counters that must be zero before the first call that uses
  *              the buffer; every completed call leaves them zero again.
  * Calls that share one workspace must not overlap on the GPU.
- * Paths: M <= 2 runs the decode-sized GEMV kernel (no workspace) where its
- * plan fits; 3 <= M <= 5 with K a multiple of 512 runs the narrow-row kernel
+ * Paths (B in {2,3,4}): M <= 2 runs the decode-sized GEMV kernel (no
+ * workspace) where its plan fits; 3 <= M <= 5 with K a multiple of 512 runs
+ * the narrow-row kernel
  * ([CQ] "压缩权重必须“边解码、边计算”": the narrow-row GEMV; register-operand
  * tensor-core MMAs, 16-row x one-slice work units split evenly over the SMs,
  * row blocks shared by two CTAs summed through the workspace), also the
  * fallback of M <= 2 shapes the GEMV does not take; everything else
  * runs the tensor-core engine (128-row weight tiles, 16- to 192-token
  * activation tiles, stream-K over the K slices, partial tiles summed in a
- * fixed order).  Results are run-to-run deterministic.  All three kernels
+ * fixed order).  B in {1,5,6,7,8} always runs the engine, with token tiles
+ * of at most 128 and a decoder that evaluates each code's level (FP64 q(t)
+ * times s, rounded to FP32 and then to BF16, as the pair tables of the other
+ * widths hold it) instead of looking it up.  Results are run-to-run
+ * deterministic.  All three kernels
  * are launched with programmatic dependent launch: their setup may overlap
  * the end of the preceding kernel in the stream, and they read no caller
  * memory before that kernel has completed (stream order holds).

@@ -89,8 +89,9 @@ def test_gemm_rejects_bad_arguments(lib):
         return lib.cq_gemm(a["x"], a["M"], a["packed"], a["scales"], a["ab"], a["N"], a["K"],
                            a["B"], a["G"], a["mode"], a["epi"], a["dt"], a["y"], a["ws"],
                            a["wsb"], a["s"])
-    assert call(B=1) == 2                     # the GEMM paths take B in {2, 3, 4}
-    assert call(B=5) == 2
+    assert call(B=0) == 2                     # cq_gemm takes B in 1..8
+    assert call(B=9) == 2
+    assert call(B=1, mode=1) == 2             # the midtread grid needs B >= 2
     assert call(G=192) == 2
     assert call(K=640, G=256) == 2
     assert call(M=-1) == 1
@@ -118,7 +119,7 @@ def test_gemm_noalloc_rejects_bad_arguments_before_touching_the_gpu(lib):
         a.update(kw)
         return f(a["x"], a["M"], a["packed"], a["scales"], a["ab"], a["N"], a["K"], a["B"],
                  a["G"], a["mode"], a["epi"], a["dt"], a["y"], a["s"])
-    assert call(B=5) == 2
+    assert call(B=9) == 2
     assert call(dt=2) == 1
     assert call(epi=3) == 1
     assert call(y=None) == 1

@@ -182,6 +182,48 @@ def test_gemv_small(cq, M, N, K, B, G, mode, epi, dt):
     test_gemm_small(cq, M, N, K, B, G, mode, epi, dt)
 
 
+# Code widths 1 and 5..8 ([CQ] "为什么只用两个形状参数？": the code stream is an
+# ordinary 1..8-bit integer stream; the H200 crossover section measures W5 and
+# W8): the engine's wide-code decoder at decode and prefill sizes, every width,
+# both grids, ragged N and M, several groups per row, SwiGLU and BF16 output,
+# the 128-byte swizzled rows of W8 and the unswizzled 80/96/112-byte rows.
+WIDE_CASES = [
+    # M,   N,    K,    B, G,   mode, epi, dtype
+    (1,   256,  1024, 8, 128, 0, 0, 0),
+    (2,   200,  1536, 5, 512, 0, 0, 0),
+    (1,   384,  512,  1, 128, 0, 0, 0),
+    (4,   512,  1024, 6, 256, 1, 1, 0),
+    (16,  300,  2048, 7, 512, 0, 0, 1),
+    (33,  256,  1024, 8, 256, 1, 0, 0),
+    (64,  640,  768,  5, 128, 1, 0, 0),
+    (130, 384,  1024, 6, 512, 0, 0, 0),
+    (300, 256,  1536, 8, 512, 0, 1, 1),
+    (200, 129,  512,  7, 128, 1, 0, 0),
+    (17,  1152, 3072, 1, 512, 0, 1, 0),
+]
+
+
+@pytest.mark.parametrize("M,N,K,B,G,mode,epi,dt", WIDE_CASES)
+def test_gemm_wide_codes(cq, M, N, K, B, G, mode, epi, dt):
+    test_gemm_small(cq, M, N, K, B, G, mode, epi, dt)
+
+
+@pytest.mark.parametrize("B,mode", [(5, 0), (6, 1), (7, 0), (8, 1), (1, 0)])
+def test_wide_gemm_matches_decoded_bf16_matmul(cq, B, mode):
+    """The wide-code decoder's operand is cq_decode's BF16 value: the GEMM
+    equals a matmul of cq_decode's BF16 output up to FP32 summation order."""
+    M, N, K, G = 40, 256, 1024, 256
+    codes, s, ab = make_matrix(("wide_bf16mm", B, mode), N, K, B, G, mode)
+    pk, sd, abd = to_dev(codes, s, ab, B, cq)
+    x = synthetic.activations(23 + B, M, K).cuda()
+    y = cq.cq_gemm(x, pk, sd, abd, N, K, B, G, mode).double()
+    w = cq.cq_decode(pk, sd, abd, K, B, G, mode, cq.BF16).double()
+    ref = x.double() @ w.T
+    bound = x.double().abs() @ w.abs().T
+    assert torch.all((y - ref).abs() <= 1e-5 * bound + 1e-7)
+    assert cq.device_error() == (0, 0)
+
+
 @pytest.mark.parametrize("M", [1, 2])
 def test_gemv_is_deterministic_and_cleans_workspace(cq, M):
     N, K, B, G = 7168, 3072, 3, 512
