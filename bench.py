@@ -75,7 +75,7 @@ NOMINAL_BF16_TFLOPS = 2250.0      # dense BF16 datasheet figure
 KERNEL_SOURCES = ("cq_gemv.cuh", "cq_gemv_launch.cuh", "cq_device.cuh")
 TRAFFIC = {
     "down_m1": {"kernel": "gemv_kernel<3,1>", "bytes": 8652544,
-                "sources_sha256": "253d37378681b15642e356880ad836961361511f58456029e3494acf30f3b2bb"},
+                "sources_sha256": "4bc21cfec1c73681d65a8f2cb03f13c3d0e85f9274f572aa73c0908e38002910"},
 }
 
 
@@ -116,7 +116,7 @@ def dominant_kernel(name):
         return f"quant_rows_kernel + engine_a8_kernel<{nt},{64 if B == 3 else 16}>"
     if M <= 2:
         return f"gemv_kernel<{B},{M}>"
-    if M <= 5 and K % 512 == 0:
+    if M <= 8 and K % 512 == 0 and 2 <= B <= 4:
         return f"narrow_kernel<{B},8>"
     if M <= 128:
         nt = 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128

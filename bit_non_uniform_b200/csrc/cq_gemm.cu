@@ -64,10 +64,11 @@ static GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int B, int epilogue, 
 // tensor-core engine.  (The test hook may force one of them.)
 enum GemmPath { PATH_AUTO = 0, PATH_NARROW = 1, PATH_GEMV = 2, PATH_ENGINE = 3 };
 
-// The narrow-row kernel takes 3 <= M <= 5 on its own: the GEMV is faster for
-// M <= 2 and the engine from about M = 6 (down_proj 7168 x 3072 W3 and
-// gate_up 6144 x 7168 W2, graphs of launches over weights larger than L2).
-constexpr int64_t kNrAutoMinM = 3, kNrAutoMaxM = 5;
+// The narrow-row kernel takes 3 <= M <= 8 on its own: the GEMV is faster for
+// M <= 2, and past 8 tokens (two MMAs per step) the engine is (down_proj
+// 7168 x 3072 W3 at M = 8: 18.2 against 20.3 us; gate_up 6144 x 7168 W2:
+// 28.0 against 27.7 us; graphs of launches over weights larger than L2).
+constexpr int64_t kNrAutoMinM = 3, kNrAutoMaxM = 8;
 static bool narrow_wanted(int64_t M, int path) {
   return path == PATH_NARROW || (path == PATH_AUTO && M >= kNrAutoMinM && M <= kNrAutoMaxM);
 }

@@ -122,7 +122,7 @@ CQ_API int cq_decode(const uint8_t *packed, const float *scales, const uint16_t 
  *              the buffer; every completed call leaves them zero again.
  * Calls that share one workspace must not overlap on the GPU.
  * Paths (B in {2,3,4}): M <= 2 runs the decode-sized GEMV kernel (no
- * workspace) where its plan fits; 3 <= M <= 5 with K a multiple of 512 runs
+ * workspace) where its plan fits; 3 <= M <= 8 with K a multiple of 512 runs
  * the narrow-row kernel
  * ([CQ] "压缩权重必须“边解码、边计算”": the narrow-row GEMV; register-operand
  * tensor-core MMAs, 16-row x one-slice work units split evenly over the SMs,
