@@ -3,6 +3,8 @@
 // engine launches (gate/up + SwiGLU, down) and the weighted combine.
 #include <cuda_runtime.h>
 
+#include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "cq.h"
@@ -318,21 +320,51 @@ static bool moe_gemv_plan(const MoePlan& m, int64_t T, int k, int E, int64_t H, 
   return true;
 }
 
+// Experts may mix bit widths: 64-entry pair tables (any of 2, 3, 4 bits), or
+// the wide-code decoder when the layer has a width outside {2, 3, 4}.
 template <int NT>
-static int launch_grouped(const EngineParams& p, const CUtensorMap& xmap, cudaStream_t s) {
+static int launch_grouped(const EngineParams& p, const CUtensorMap& xmap, bool wide,
+                          cudaStream_t s) {
   CUtensorMap unused;
   memset(&unused, 0, sizeof(unused));
-  return launch_engine<NT, 64>(p, xmap, unused, s);   // experts may mix bit widths
+  if (wide) return launch_engine<NT, 0>(p, xmap, unused, s);
+  return launch_engine<NT, 64>(p, xmap, unused, s);
 }
 
-static int launch_grouped_nt(int NT, const EngineParams& p, const CUtensorMap& xmap,
+static int launch_grouped_nt(int NT, const EngineParams& p, const CUtensorMap& xmap, bool wide,
                              cudaStream_t s) {
   switch (NT) {
-    case 16: return launch_grouped<16>(p, xmap, s);
-    case 32: return launch_grouped<32>(p, xmap, s);
-    case 64: return launch_grouped<64>(p, xmap, s);
-    default: return launch_grouped<128>(p, xmap, s);
+    case 16: return launch_grouped<16>(p, xmap, wide, s);
+    case 32: return launch_grouped<32>(p, xmap, wide, s);
+    case 64: return launch_grouped<64>(p, xmap, wide, s);
+    default: return launch_grouped<128>(p, xmap, wide, s);
   }
+}
+
+// The code widths of every layer table cq_moe_prepare_layer wrote, by the
+// table's device address: the grouped launches pick their decoder from it
+// without reading the table back.  A table it does not know is taken to hold
+// widths 2..4 only (a wider expert in it is flagged on the device).
+struct LayerWidths {
+  int bmin, bmax;
+};
+static std::mutex g_layer_mu;
+static std::unordered_map<const void*, LayerWidths> g_layer_widths;
+
+static void remember_layer(const void* layer, LayerWidths w) {
+  std::lock_guard<std::mutex> lock(g_layer_mu);
+  g_layer_widths[layer] = w;
+}
+
+static void forget_layer(const void* layer) {
+  std::lock_guard<std::mutex> lock(g_layer_mu);
+  g_layer_widths.erase(layer);
+}
+
+static LayerWidths layer_widths(const void* layer) {
+  std::lock_guard<std::mutex> lock(g_layer_mu);
+  const auto it = g_layer_widths.find(layer);
+  return it == g_layer_widths.end() ? LayerWidths{2, 4} : it->second;
 }
 
 }  // namespace cq
@@ -354,6 +386,8 @@ extern "C" int cq_moe_prepare_layer(const cq_expert_desc* experts, int E, int64_
   if (st != CQ_OK) return st;
   if (!experts || !layer) return CQ_ERR_INVALID_ARG;
   if (!aligned(layer, 64)) return CQ_ERR_UNSUPPORTED;
+  forget_layer(layer);
+  LayerWidths lw = {8, 1};
   std::vector<LayerEntry> host(static_cast<size_t>(E));
   memset(host.data(), 0, host.size() * sizeof(LayerEntry));
   std::vector<GvExpert> gvx(static_cast<size_t>(2) * E);
@@ -365,8 +399,10 @@ extern "C" int cq_moe_prepare_layer(const cq_expert_desc* experts, int E, int64_
     for (int w = 0; w < 2; ++w) {
       if (d[w]->reserved != 0) return CQ_ERR_INVALID_ARG;
       st = validate_matrix(d[w]->packed, d[w]->scales, d[w]->ab, rows[w], cols[w], d[w]->B, G,
-                           CQ_GRID_MIDRISE);
+                           CQ_GRID_MIDRISE, 1, 8);
       if (st != CQ_OK) return st;
+      lw.bmin = d[w]->B < lw.bmin ? d[w]->B : lw.bmin;
+      lw.bmax = d[w]->B > lw.bmax ? d[w]->B : lw.bmax;
       st = encode_packed_rows(&host[e].map[w], d[w]->packed, rows[w], cols[w] * d[w]->B / 8,
                               d[w]->B);
       if (st != CQ_OK) return st;
@@ -380,7 +416,7 @@ extern "C" int cq_moe_prepare_layer(const cq_expert_desc* experts, int E, int64_
       g.mat.scales = d[w]->scales;
       g.mat.ab = reinterpret_cast<const uint32_t*>(d[w]->ab);
       g.mat.B = d[w]->B;
-      if (G / 8 * d[w]->B <= 256) {
+      if (d[w]->B >= 2 && d[w]->B <= 4 && G / 8 * d[w]->B <= 256) {
         const int ng = static_cast<int>(cols[w] / G);
         st = encode_packed_gemv(&g.map, d[w]->packed, rows[w], cols[w], d[w]->B, G,
                                 w == 0 ? CQ_EPI_SWIGLU : CQ_EPI_NONE, ng % 2 == 0 ? 2 : 1);
@@ -394,6 +430,7 @@ extern "C" int cq_moe_prepare_layer(const cq_expert_desc* experts, int E, int64_
   if (cudaMemcpy(static_cast<uint8_t*>(layer) + gv_table_offset(E), gvx.data(),
                  gvx.size() * sizeof(GvExpert), cudaMemcpyHostToDevice) != cudaSuccess)
     return CQ_ERR_CUDA;
+  remember_layer(layer, lw);
   return CQ_OK;
 }
 
@@ -419,6 +456,9 @@ extern "C" int cq_moe_grouped_gemm(const uint16_t* tokens, int64_t T, const int3
   if (!aligned(tokens, 16) || !aligned(layer, 64) || !aligned(workspace, 256) ||
       (route_out && !aligned(route_out, 16)) || (out && !aligned(out, 16)))
     return CQ_ERR_UNSUPPORTED;
+  const LayerWidths lw = layer_widths(layer);
+  const bool wide = lw.bmin < 2 || lw.bmax > 4;
+  if (grid_mode == CQ_GRID_MIDTREAD && lw.bmin < 2) return CQ_ERR_UNSUPPORTED;
   const int sms = num_sms();
   if (sms <= 0) return CQ_ERR_CUDA;
   const MoePlan m = moe_plan(T, k, E, H, I, sms);
@@ -449,7 +489,7 @@ extern "C" int cq_moe_grouped_gemm(const uint16_t* tokens, int64_t T, const int3
     return CQ_ERR_CUDA;
   // decode-sized layers (few routes per expert) take the grouped GEMV path
   MoeGvParams gvp[2];
-  const bool gv = moe_gemv_plan(m, T, k, E, H, I, G, grid_mode, sms, gvp);
+  const bool gv = !wide && moe_gemv_plan(m, T, k, E, H, I, G, grid_mode, sms, gvp);
   const GvExpert* gvx = reinterpret_cast<const GvExpert*>(
       static_cast<const uint8_t*>(layer) + gv_table_offset(E));
   int* chunks = reinterpret_cast<int*>(ws + m.o_chunks);
@@ -517,7 +557,7 @@ extern "C" int cq_moe_grouped_gemm(const uint16_t* tokens, int64_t T, const int3
     p.partial_slots = 2 * m.P;
     p.counter_len = static_cast<int>((which == 0 ? m.n_rt_gu : m.n_rt_dn) * m.max_tt);
     p.timeout_ns = kDefaultTimeoutNs;
-    st = launch_grouped_nt(m.NT, p, which == 0 ? xmap_gu : xmap_dn, s);
+    st = launch_grouped_nt(m.NT, p, which == 0 ? xmap_gu : xmap_dn, wide, s);
     if (st != CQ_OK) return st;
   }
   // 5. weighted combine (and clearing of dropped routes' rows)

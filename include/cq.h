@@ -34,10 +34,10 @@
  *     NULL = legacy default stream) and returns a cq_status.  Arguments are
  *     validated on the host before anything is launched; on error nothing
  *     is launched and no output is touched.
- *   - Supported: B in 1..8 for cq_pack, cq_decode, cq_gemm and
- *     cq_gemm_noalloc (midtread: 2..8; the 8-bit code stream of [CQ]
- *     "为什么只用两个形状参数？" is an ordinary 1..8-bit integer stream);
- *     B in {2,3,4} for the MoE layer and the Dynamic A8 path;
+ *   - Supported: B in 1..8 for cq_pack, cq_decode, cq_gemm,
+ *     cq_gemm_noalloc and the MoE layer (midtread: 2..8; the code stream of
+ *     [CQ] "为什么只用两个形状参数？" is an ordinary 1..8-bit integer stream);
+ *     B in {2,3,4} for the Dynamic A8 path;
  *     G a multiple of 128; K a multiple of G;
  *     N >= 1; packed / x / y / workspace 16-byte aligned; scales and ab
  *     4-byte aligned.
@@ -234,8 +234,14 @@ typedef struct {
  * of E descriptions (device pointers inside); `layer` is device memory of
  * cq_moe_layer_bytes(E) bytes owned by the caller, valid as long as the
  * expert weights do not move.  Synchronous (run once per layer, at load).
- * Each matrix must satisfy the cq_gemm requirements (B in {2,3,4},
+ * Each matrix must satisfy the cq_gemm requirements (B in 1..8,
  * G % 128 == 0, H and I multiples of G, I % 64 == 0, packed 16-byte aligned).
+ * The library remembers, by the table's address, the widths written there:
+ * cq_moe_grouped_gemm takes a layer with a width outside {2,3,4} through the
+ * tensor-core engine's wide-code decoder (and never the decode-sized path),
+ * so such a table must be used at the address this call wrote; a copy of it
+ * elsewhere is taken to hold widths 2..4 only, and its wider experts are
+ * flagged on the device (cq_get_device_error) instead of computed.
  */
 CQ_API size_t cq_moe_layer_bytes(int E);
 CQ_API int cq_moe_prepare_layer(const cq_expert_desc *experts, int E, int64_t H, int64_t I,
@@ -259,7 +265,8 @@ CQ_API int cq_moe_prepare_layer(const cq_expert_desc *experts, int E, int64_t H,
  *   route_out  float [T*k][H] per-route outputs y_r (may be NULL)
  *   out        [T][H] combined output in out_dtype (may be NULL)
  *   workspace  device scratch of at least cq_moe_workspace_size(...) bytes
- * Calls that share one workspace must not overlap on the GPU.
+ * Calls that share one workspace must not overlap on the GPU.  A layer with
+ * a 1-bit expert returns CQ_ERR_UNSUPPORTED on the midtread grid.
  */
 CQ_API size_t cq_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I, int G);
 CQ_API int cq_moe_grouped_gemm(const uint16_t *tokens, int64_t T, const int32_t *topk_ids,

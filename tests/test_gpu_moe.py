@@ -140,6 +140,11 @@ TOY = [
     # experts with one, two and more routes (chunks of two)
     (512, 256, 32, 24, 2, 128, (2, 3, 4), "uniform"),
     (1024, 512, 16, 24, 2, 512, (3, 4), "zipf"),
+    # code widths 1 and 5..8 beside the table widths ([CQ] "为什么只用两个形状参数？":
+    # an ordinary 1..8-bit code stream): the whole layer takes the engine's
+    # wide-code decoder, at prefill and at decode sizes
+    (512, 256, 8, 37, 2, 128, (5, 8, 2, 3), "uniform"),
+    (512, 256, 16, 12, 2, 256, (1, 6, 7, 4), "uniform"),
 ]
 
 
