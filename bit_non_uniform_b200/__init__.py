@@ -75,6 +75,8 @@ def lib():
         "cq_moe_grouped_gemm": (i32, [P, i64, P, P, i32, i32, P, i64, i64, i32, i32, i32,
                                       P, P, P, sz, P]),
         "cq_gemm_noalloc": (i32, [P, i64, P, P, P, i64, i64, i32, i32, i32, i32, i32, P, P]),
+        "cq_gemm_host": (i32, [P, i64, P, P, P, i64, i64, i32, i32, i32, i32, i32, P, P, P, P,
+                               sz, P]),
         "cq_get_device_error": (i32, [P, ctypes.POINTER(ctypes.c_int)]),
         "cq_test_gemm_bounded": (i32, [P, i64, P, P, P, i64, i64, i32, i32, P, P, sz, u64,
                                        i32, P]),
@@ -190,6 +192,34 @@ def gemm_on_path(path: int, x, packed, scales, ab, N: int, K: int, B: int, G: in
                                    mode, epilogue, out_dtype, _ptr(out), _ptr(ws), ws.numel(),
                                    path, _stream(stream)), "cq_test_gemm_path")
     return out
+
+
+def cq_gemm_host(x_host, packed, scales, ab, N: int, K: int, B: int, G: int,
+                 mode: int = MIDRISE, epilogue: int = EPI_NONE, out_dtype: int = F32,
+                 y_host=None, x_dev=None, y_dev=None, workspace=None, stream=None):
+    """cq_gemm with x and y in host memory (pinned CPU tensors keep the
+    copies asynchronous): the copies and the GEMM are queued on `stream`;
+    synchronize it before reading y_host."""
+    _need_cuda(packed, scales, ab)
+    assert x_host.device.type == "cpu" and x_host.dtype == torch.bfloat16
+    assert x_host.is_contiguous()
+    M = x_host.shape[0]
+    dev = packed.device
+    ncol = N // 2 if epilogue == EPI_SWIGLU else N
+    dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+    if y_host is None:
+        y_host = torch.empty((M, ncol), dtype=dt).pin_memory()
+    if x_dev is None:
+        x_dev = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    if y_dev is None:
+        y_dev = torch.empty((M, ncol), dtype=dt, device=dev)
+    if workspace is None:
+        workspace = gemm_workspace(M, N, K, B, G, epilogue, dev)
+    _check(lib().cq_gemm_host(x_host.data_ptr(), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K,
+                              B, G, mode, epilogue, out_dtype, y_host.data_ptr(), _ptr(x_dev),
+                              _ptr(y_dev), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "cq_gemm_host")
+    return y_host
 
 
 def cq_gemm_noalloc(x, packed, scales, ab, N: int, K: int, B: int, G: int,

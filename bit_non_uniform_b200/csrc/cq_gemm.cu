@@ -264,6 +264,36 @@ extern "C" int cq_gemm(const uint16_t* x, int64_t M, const uint8_t* packed, cons
                    workspace, ws_bytes, static_cast<cudaStream_t>(stream), kDefaultTimeoutNs, 0);
 }
 
+extern "C" int cq_gemm_host(const uint16_t* x_host, int64_t M, const uint8_t* packed,
+                            const float* scales, const uint16_t* ab, int64_t N, int64_t K, int B,
+                            int G, int grid_mode, int epilogue, int out_dtype, void* y_host,
+                            uint16_t* x_dev, void* y_dev, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  // every check before anything is queued
+  int st = validate_gemm(x_dev, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue,
+                         out_dtype, y_dev);
+  if (st != CQ_OK) return st;
+  if (M == 0 || N == 0) return CQ_OK;
+  if (!x_host || !y_host) return CQ_ERR_INVALID_ARG;
+  int sms = num_sms();
+  if (sms <= 0) return CQ_ERR_CUDA;
+  const size_t need = gemm_workspace_size(M, N, K, B, G, epilogue, sms);
+  if (ws_bytes < need || (need && !workspace)) return CQ_ERR_WORKSPACE;
+  if (need && !aligned(workspace, 16)) return CQ_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t x_bytes = static_cast<size_t>(M) * K * 2;
+  const int64_t ncol = epilogue == CQ_EPI_SWIGLU ? N / 2 : N;
+  const size_t y_bytes = static_cast<size_t>(M) * ncol * (out_dtype == CQ_DTYPE_BF16 ? 2 : 4);
+  if (cudaMemcpyAsync(x_dev, x_host, x_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return CQ_ERR_CUDA;
+  st = gemm_impl(x_dev, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype, y_dev,
+                 workspace, ws_bytes, s, kDefaultTimeoutNs, 0);
+  if (st != CQ_OK) return st;
+  if (cudaMemcpyAsync(y_host, y_dev, y_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return CQ_ERR_CUDA;
+  return CQ_OK;
+}
+
 // Profiling hook (declared in cq_hooks.h): cq_gemm that also writes per-CTA
 // event timestamps to trace ([grid][64] uint64 words of device memory).
 extern "C" CQ_API int cq_trace_gemm(const uint16_t* x, int64_t M, const uint8_t* packed,

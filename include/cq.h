@@ -175,6 +175,30 @@ CQ_API int cq_gemm_noalloc(const uint16_t *x, int64_t M, const uint8_t *packed,
                            void *stream);
 
 /*
+ * cq_gemm_host -- cq_gemm for a caller whose activations and outputs live in
+ * HOST memory (one decode step served from the host): queues on `stream`
+ * the copy of x_host into the device staging buffer x_dev, cq_gemm on it,
+ * and the copy of the output from the device staging buffer y_dev into
+ * y_host.  Same arguments, semantics and results as cq_gemm otherwise (the
+ * article has no counterpart; this is a calling convenience).
+ *   x_host  HOST bfloat16 [M][K]; y_host HOST [M][N] (or [M][N/2] with
+ *           SwiGLU) in out_dtype.  Page-locked (pinned) host buffers keep
+ *           the copies asynchronous; pageable ones make the driver stage
+ *           them synchronously.  Both must stay valid until the stream has
+ *           run the call's work.
+ *   x_dev   DEVICE staging buffer of M*K*2 bytes; y_dev DEVICE staging
+ *           buffer of the output's size; both 16-byte aligned, owned by the
+ *           caller (the library allocates nothing).
+ *   workspace / ws_bytes as cq_gemm (cq_gemm_workspace_size bytes).
+ * Every argument and size check runs before anything is queued.
+ */
+CQ_API int cq_gemm_host(const uint16_t *x_host, int64_t M, const uint8_t *packed,
+                        const float *scales, const uint16_t *ab, int64_t N, int64_t K, int B,
+                        int G, int grid_mode, int epilogue, int out_dtype, void *y_host,
+                        uint16_t *x_dev, void *y_dev, void *workspace, size_t ws_bytes,
+                        void *stream);
+
+/*
  * Dynamic A8 ([CQ] "一份 checkpoint，同时服务 A16 与 Dynamic A8"): the same
  * checkpoint served with INT8 activations.  The article's carrier and
  * activation formulas were lost in extraction; this library reads them as

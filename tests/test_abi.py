@@ -104,6 +104,32 @@ def test_gemm_rejects_bad_arguments(lib):
     assert call(N=0) == 0
 
 
+def test_gemm_host_rejects_bad_arguments_before_touching_the_gpu(lib):
+    """The argument checks of cq_gemm_host run before any copy is queued:
+    on a machine without a GPU these calls return their status."""
+    f = lib.cq_gemm_host
+    P = ctypes.c_void_p
+    f.argtypes = [P, ctypes.c_int64, P, P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P,
+                  ctypes.c_size_t, P]
+
+    def call(**kw):
+        a = dict(xh=FAKE, M=4, packed=FAKE, scales=FAKE, ab=FAKE, N=256, K=512, B=3, G=128,
+                 mode=0, epi=0, dt=0, yh=FAKE, xd=FAKE, yd=FAKE, ws=FAKE, wsb=1 << 30, s=None)
+        a.update(kw)
+        return f(a["xh"], a["M"], a["packed"], a["scales"], a["ab"], a["N"], a["K"], a["B"],
+                 a["G"], a["mode"], a["epi"], a["dt"], a["yh"], a["xd"], a["yd"], a["ws"],
+                 a["wsb"], a["s"])
+    assert call(B=9) == 2
+    assert call(dt=2) == 1
+    assert call(epi=3) == 1
+    assert call(yd=None) == 1
+    assert call(xd=FAKE_ODD) == 2
+    assert call(M=-1) == 1
+    assert call(epi=1, N=200) == 2
+    assert call(M=0) == 0
+
+
 def test_gemm_noalloc_rejects_bad_arguments_before_touching_the_gpu(lib):
     """Every check runs before the fixed array is looked up or cleared: on a
     machine without a GPU these calls return their status without a CUDA

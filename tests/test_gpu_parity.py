@@ -320,6 +320,32 @@ def check_swiglu(y_gpu, yr, bd, dt):
     assert not (err > tol).any(), f"swiglu: worst ratio {np.max(err / tol):.3f}"
 
 
+@pytest.mark.parametrize("M,N,K,B,G,epi,dt,pinned", [
+    (1, 7168, 3072, 3, 512, 0, 0, True),
+    (2, 512, 2048, 4, 256, 1, 1, True),
+    (5, 640, 1024, 2, 512, 0, 0, False),
+    (16, 384, 1024, 8, 128, 0, 1, True),
+    (300, 256, 1536, 3, 512, 1, 0, True),
+])
+def test_gemm_host_buffers_equal_device_call(cq, M, N, K, B, G, epi, dt, pinned):
+    """cq_gemm_host (x and y in host memory, copies queued on the stream)
+    gives exactly cq_gemm's output: the kernels are run-to-run deterministic."""
+    codes, s, ab = make_matrix(("host", M, N, B), N, K, B, G)
+    pk, sd, abd = to_dev(codes, s, ab, B, cq)
+    x = synthetic.activations(41 + M, M, K)
+    ref = cq.cq_gemm(x.cuda(), pk, sd, abd, N, K, B, G, 0, epi, dt)
+    xh = x.pin_memory() if pinned else x.clone()
+    ncol = N // 2 if epi else N
+    yh = torch.empty((M, ncol), dtype=torch.float32 if dt == 0 else torch.bfloat16)
+    if pinned:
+        yh = yh.pin_memory()
+    st = torch.cuda.Stream()
+    got = cq.cq_gemm_host(xh, pk, sd, abd, N, K, B, G, 0, epi, dt, y_host=yh, stream=st)
+    st.synchronize()
+    assert torch.equal(got, ref.cpu())
+    assert cq.device_error() == (0, 0)
+
+
 def test_gemm_is_deterministic_and_cleans_workspace(cq):
     M, N, K, B, G = 7, 896, 3072, 3, 512
     codes, s, ab = make_matrix(("det",), N, K, B, G)
