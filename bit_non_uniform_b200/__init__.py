@@ -14,6 +14,7 @@ The calls mirror ``include/cq.h``:
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -99,6 +100,13 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _on_stream(stream=None):
+    """Allocations and fills of a binding call go on the call's stream, so
+    that the buffers it creates are ready (and are recycled) in that
+    stream's order."""
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+
+
 def _stream(stream=None):
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
@@ -121,25 +129,27 @@ def version() -> int:
 
 def cq_pack(codes: torch.Tensor, B: int, out: torch.Tensor | None = None, stream=None):
     """codes uint8 [N][K] (CUDA) -> packed uint8 [N][K*B/8]."""
-    _need_cuda(codes)
-    codes = codes.contiguous()
-    N, K = codes.shape
-    if out is None:
-        out = torch.empty((N, K * B // 8), dtype=torch.uint8, device=codes.device)
-    _check(lib().cq_pack(_ptr(codes), N, K, B, _ptr(out), _stream(stream)), "cq_pack")
-    return out
+    with _on_stream(stream):
+        _need_cuda(codes)
+        codes = codes.contiguous()
+        N, K = codes.shape
+        if out is None:
+            out = torch.empty((N, K * B // 8), dtype=torch.uint8, device=codes.device)
+        _check(lib().cq_pack(_ptr(codes), N, K, B, _ptr(out), _stream(stream)), "cq_pack")
+        return out
 
 
 def cq_decode(packed, scales, ab, K: int, B: int, G: int, mode: int = MIDRISE,
               out_dtype: int = F32, stream=None):
     """Decode packed codes + (s, a, b) into W [N][K] (float32 or bfloat16)."""
-    _need_cuda(packed, scales, ab)
-    N = packed.shape[0]
-    dt = torch.float32 if out_dtype == F32 else torch.bfloat16
-    W = torch.empty((N, K), dtype=dt, device=packed.device)
-    _check(lib().cq_decode(_ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G, mode, out_dtype,
-                           _ptr(W), _stream(stream)), "cq_decode")
-    return W
+    with _on_stream(stream):
+        _need_cuda(packed, scales, ab)
+        N = packed.shape[0]
+        dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+        W = torch.empty((N, K), dtype=dt, device=packed.device)
+        _check(lib().cq_decode(_ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G, mode, out_dtype,
+                               _ptr(W), _stream(stream)), "cq_decode")
+        return W
 
 
 def gemm_workspace_size(M, N, K, B, G, epilogue=EPI_NONE) -> int:
@@ -156,20 +166,21 @@ def cq_gemm(x, packed, scales, ab, N: int, K: int, B: int, G: int, mode: int = M
             epilogue: int = EPI_NONE, out_dtype: int = F32, workspace=None, out=None,
             stream=None):
     """y = x W^T with W given packed; x bfloat16 [M][K]."""
-    _need_cuda(x, packed, scales, ab)
-    assert x.dtype == torch.bfloat16 and x.is_contiguous()
-    M = x.shape[0]
-    ncol = N // 2 if epilogue == EPI_SWIGLU else N
-    if out is None:
-        dt = torch.float32 if out_dtype == F32 else torch.bfloat16
-        out = torch.empty((M, ncol), dtype=dt, device=x.device)
-    if workspace is None:
-        workspace = gemm_workspace(M, N, K, B, G, epilogue, x.device)
-    _check(lib().cq_gemm(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G, mode,
-                         epilogue, out_dtype, _ptr(out), _ptr(workspace),
-                         workspace.numel() * workspace.element_size(), _stream(stream)),
-           "cq_gemm")
-    return out
+    with _on_stream(stream):
+        _need_cuda(x, packed, scales, ab)
+        assert x.dtype == torch.bfloat16 and x.is_contiguous()
+        M = x.shape[0]
+        ncol = N // 2 if epilogue == EPI_SWIGLU else N
+        if out is None:
+            dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+            out = torch.empty((M, ncol), dtype=dt, device=x.device)
+        if workspace is None:
+            workspace = gemm_workspace(M, N, K, B, G, epilogue, x.device)
+        _check(lib().cq_gemm(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G, mode,
+                             epilogue, out_dtype, _ptr(out), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)),
+               "cq_gemm")
+        return out
 
 
 # kernels of cq_gemm (test hook cq_test_gemm_path)
@@ -181,17 +192,18 @@ def gemm_on_path(path: int, x, packed, scales, ab, N: int, K: int, B: int, G: in
                  stream=None):
     """cq_gemm on a chosen kernel (a test hook); raises CQError with status 2
     when that kernel does not take the problem."""
-    _need_cuda(x, packed, scales, ab)
-    M = x.shape[0]
-    ncol = N // 2 if epilogue == EPI_SWIGLU else N
-    dt = torch.float32 if out_dtype == F32 else torch.bfloat16
-    out = torch.empty((M, ncol), dtype=dt, device=x.device)
-    n = int(lib().cq_test_gemm_path_workspace_size(M, N, K, B, G, epilogue, path))
-    ws = torch.zeros(max(n, 16), dtype=torch.uint8, device=x.device)
-    _check(lib().cq_test_gemm_path(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G,
-                                   mode, epilogue, out_dtype, _ptr(out), _ptr(ws), ws.numel(),
-                                   path, _stream(stream)), "cq_test_gemm_path")
-    return out
+    with _on_stream(stream):
+        _need_cuda(x, packed, scales, ab)
+        M = x.shape[0]
+        ncol = N // 2 if epilogue == EPI_SWIGLU else N
+        dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+        out = torch.empty((M, ncol), dtype=dt, device=x.device)
+        n = int(lib().cq_test_gemm_path_workspace_size(M, N, K, B, G, epilogue, path))
+        ws = torch.zeros(max(n, 16), dtype=torch.uint8, device=x.device)
+        _check(lib().cq_test_gemm_path(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G,
+                                       mode, epilogue, out_dtype, _ptr(out), _ptr(ws), ws.numel(),
+                                       path, _stream(stream)), "cq_test_gemm_path")
+        return out
 
 
 def cq_gemm_host(x_host, packed, scales, ab, N: int, K: int, B: int, G: int,
@@ -200,42 +212,44 @@ def cq_gemm_host(x_host, packed, scales, ab, N: int, K: int, B: int, G: int,
     """cq_gemm with x and y in host memory (pinned CPU tensors keep the
     copies asynchronous): the copies and the GEMM are queued on `stream`;
     synchronize it before reading y_host."""
-    _need_cuda(packed, scales, ab)
-    assert x_host.device.type == "cpu" and x_host.dtype == torch.bfloat16
-    assert x_host.is_contiguous()
-    M = x_host.shape[0]
-    dev = packed.device
-    ncol = N // 2 if epilogue == EPI_SWIGLU else N
-    dt = torch.float32 if out_dtype == F32 else torch.bfloat16
-    if y_host is None:
-        y_host = torch.empty((M, ncol), dtype=dt).pin_memory()
-    if x_dev is None:
-        x_dev = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-    if y_dev is None:
-        y_dev = torch.empty((M, ncol), dtype=dt, device=dev)
-    if workspace is None:
-        workspace = gemm_workspace(M, N, K, B, G, epilogue, dev)
-    _check(lib().cq_gemm_host(x_host.data_ptr(), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K,
-                              B, G, mode, epilogue, out_dtype, y_host.data_ptr(), _ptr(x_dev),
-                              _ptr(y_dev), _ptr(workspace), workspace.numel(), _stream(stream)),
-           "cq_gemm_host")
-    return y_host
+    with _on_stream(stream):
+        _need_cuda(packed, scales, ab)
+        assert x_host.device.type == "cpu" and x_host.dtype == torch.bfloat16
+        assert x_host.is_contiguous()
+        M = x_host.shape[0]
+        dev = packed.device
+        ncol = N // 2 if epilogue == EPI_SWIGLU else N
+        dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+        if y_host is None:
+            y_host = torch.empty((M, ncol), dtype=dt).pin_memory()
+        if x_dev is None:
+            x_dev = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        if y_dev is None:
+            y_dev = torch.empty((M, ncol), dtype=dt, device=dev)
+        if workspace is None:
+            workspace = gemm_workspace(M, N, K, B, G, epilogue, dev)
+        _check(lib().cq_gemm_host(x_host.data_ptr(), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K,
+                                  B, G, mode, epilogue, out_dtype, y_host.data_ptr(), _ptr(x_dev),
+                                  _ptr(y_dev), _ptr(workspace), workspace.numel(), _stream(stream)),
+               "cq_gemm_host")
+        return y_host
 
 
 def cq_gemm_noalloc(x, packed, scales, ab, N: int, K: int, B: int, G: int,
                     mode: int = MIDRISE, epilogue: int = EPI_NONE, out_dtype: int = F32,
                     out=None, stream=None):
     """cq_gemm without a workspace (scratch in libcq's fixed array; M <= 16)."""
-    _need_cuda(x, packed, scales, ab)
-    M = x.shape[0]
-    ncol = N // 2 if epilogue == EPI_SWIGLU else N
-    if out is None:
-        dt = torch.float32 if out_dtype == F32 else torch.bfloat16
-        out = torch.empty((M, ncol), dtype=dt, device=x.device)
-    _check(lib().cq_gemm_noalloc(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G,
-                                 mode, epilogue, out_dtype, _ptr(out), _stream(stream)),
-           "cq_gemm_noalloc")
-    return out
+    with _on_stream(stream):
+        _need_cuda(x, packed, scales, ab)
+        M = x.shape[0]
+        ncol = N // 2 if epilogue == EPI_SWIGLU else N
+        if out is None:
+            dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+            out = torch.empty((M, ncol), dtype=dt, device=x.device)
+        _check(lib().cq_gemm_noalloc(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G,
+                                     mode, epilogue, out_dtype, _ptr(out), _stream(stream)),
+               "cq_gemm_noalloc")
+        return out
 
 
 def gemm_a8_workspace_size(M, N, K, B, G, epilogue=EPI_NONE) -> int:
@@ -244,34 +258,36 @@ def gemm_a8_workspace_size(M, N, K, B, G, epilogue=EPI_NONE) -> int:
 
 def cq_quant_rows(x, stream=None):
     """Per-row dynamic INT8 quantization: (xq int8 [M][K], absmax f32 [M])."""
-    _need_cuda(x)
-    assert x.dtype == torch.bfloat16 and x.is_contiguous()
-    M, K = x.shape
-    xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
-    absmax = torch.empty(M, dtype=torch.float32, device=x.device)
-    _check(lib().cq_quant_rows(_ptr(x), M, K, _ptr(xq), _ptr(absmax), _stream(stream)),
-           "cq_quant_rows")
-    return xq, absmax
+    with _on_stream(stream):
+        _need_cuda(x)
+        assert x.dtype == torch.bfloat16 and x.is_contiguous()
+        M, K = x.shape
+        xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+        absmax = torch.empty(M, dtype=torch.float32, device=x.device)
+        _check(lib().cq_quant_rows(_ptr(x), M, K, _ptr(xq), _ptr(absmax), _stream(stream)),
+               "cq_quant_rows")
+        return xq, absmax
 
 
 def cq_gemm_a8(x, packed, scales, ab, N: int, K: int, B: int, G: int, mode: int = MIDRISE,
                epilogue: int = EPI_NONE, out_dtype: int = F32, out=None, workspace=None,
                stream=None):
     """Dynamic-A8 y = x W^T: x quantized per row to INT8 inside the call."""
-    _need_cuda(x, packed, scales, ab)
-    assert x.dtype == torch.bfloat16 and x.is_contiguous()
-    M = x.shape[0]
-    ncol = N // 2 if epilogue == EPI_SWIGLU else N
-    if out is None:
-        dt = torch.float32 if out_dtype == F32 else torch.bfloat16
-        out = torch.empty((M, ncol), dtype=dt, device=x.device)
-    if workspace is None:
-        n = gemm_a8_workspace_size(M, N, K, B, G, epilogue)
-        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=x.device)
-    _check(lib().cq_gemm_a8(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G, mode,
-                            epilogue, out_dtype, _ptr(out), _ptr(workspace),
-                            workspace.numel(), _stream(stream)), "cq_gemm_a8")
-    return out
+    with _on_stream(stream):
+        _need_cuda(x, packed, scales, ab)
+        assert x.dtype == torch.bfloat16 and x.is_contiguous()
+        M = x.shape[0]
+        ncol = N // 2 if epilogue == EPI_SWIGLU else N
+        if out is None:
+            dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+            out = torch.empty((M, ncol), dtype=dt, device=x.device)
+        if workspace is None:
+            n = gemm_a8_workspace_size(M, N, K, B, G, epilogue)
+            workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=x.device)
+        _check(lib().cq_gemm_a8(_ptr(x), M, _ptr(packed), _ptr(scales), _ptr(ab), N, K, B, G, mode,
+                                epilogue, out_dtype, _ptr(out), _ptr(workspace),
+                                workspace.numel(), _stream(stream)), "cq_gemm_a8")
+        return out
 
 
 def moe_workspace_size(T, k, E, H, I, G) -> int:
@@ -311,24 +327,25 @@ def cq_moe_grouped_gemm(tokens, topk_ids, topk_w, layer, E: int, H: int, I: int,
                         mode: int = MIDRISE, out_dtype: int = F32, route_out=True,
                         combine=True, workspace=None, stream=None):
     """Routed-expert FFN of one MoE layer.  Returns (route_out, out)."""
-    _need_cuda(tokens, topk_ids, layer)
-    T, k = topk_ids.shape
-    ro = None
-    if route_out is True:
-        ro = torch.empty((T * k, H), dtype=torch.float32, device=tokens.device)
-    elif route_out is not None and route_out is not False:
-        ro = route_out
-    out = None
-    if combine:
-        dt = torch.float32 if out_dtype == F32 else torch.bfloat16
-        out = torch.empty((T, H), dtype=dt, device=tokens.device)
-    if workspace is None:
-        workspace = moe_workspace(T, k, E, H, I, G, tokens.device)
-    _check(lib().cq_moe_grouped_gemm(
-        _ptr(tokens), T, _ptr(topk_ids), _ptr(topk_w) if topk_w is not None else None, k, E,
-        _ptr(layer), H, I, G, mode, out_dtype, _ptr(ro), _ptr(out), _ptr(workspace),
-        workspace.numel(), _stream(stream)), "cq_moe_grouped_gemm")
-    return ro, out
+    with _on_stream(stream):
+        _need_cuda(tokens, topk_ids, layer)
+        T, k = topk_ids.shape
+        ro = None
+        if route_out is True:
+            ro = torch.empty((T * k, H), dtype=torch.float32, device=tokens.device)
+        elif route_out is not None and route_out is not False:
+            ro = route_out
+        out = None
+        if combine:
+            dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+            out = torch.empty((T, H), dtype=dt, device=tokens.device)
+        if workspace is None:
+            workspace = moe_workspace(T, k, E, H, I, G, tokens.device)
+        _check(lib().cq_moe_grouped_gemm(
+            _ptr(tokens), T, _ptr(topk_ids), _ptr(topk_w) if topk_w is not None else None, k, E,
+            _ptr(layer), H, I, G, mode, out_dtype, _ptr(ro), _ptr(out), _ptr(workspace),
+            workspace.numel(), _stream(stream)), "cq_moe_grouped_gemm")
+        return ro, out
 
 
 def device_error(stream=None) -> tuple[int, int]:
