@@ -264,6 +264,61 @@ extern "C" int cq_gemm(const uint16_t* x, int64_t M, const uint8_t* packed, cons
                    workspace, ws_bytes, static_cast<cudaStream_t>(stream), kDefaultTimeoutNs, 0);
 }
 
+// ---------------------------------------------------------------------------
+// host-buffer GEMM: copies between page-locked host memory and the device
+// staging buffers as kernels chained to the GEMM by programmatic dependent
+// launch (a copy-engine transfer between two kernels breaks the chain and
+// adds its own start latency on each side)
+// ---------------------------------------------------------------------------
+constexpr int kCopyThreads = 256;
+
+// dst[0, bytes) = src[0, bytes); both 16-byte aligned.  Waits for the
+// preceding grid before writing (the previous GEMM may still read dst, or
+// the GEMM this copy follows may still write src).
+__global__ void __launch_bounds__(kCopyThreads)
+    host_copy_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, int64_t bytes) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int64_t n16 = bytes >> 4;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kCopyThreads;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kCopyThreads + threadIdx.x; i < n16;
+       i += stride)
+    reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(src)[i];
+  if (blockIdx.x == 0 && threadIdx.x < (bytes & 15))
+    dst[n16 * 16 + threadIdx.x] = src[n16 * 16 + threadIdx.x];
+}
+
+static int launch_host_copy(const void* src, void* dst, int64_t bytes, int sms, cudaStream_t s) {
+  if (bytes <= 0) return CQ_OK;
+  const int64_t n16 = (bytes + 15) >> 4;
+  int64_t blocks = (n16 + kCopyThreads - 1) / kCopyThreads;
+  if (blocks > sms) blocks = sms;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(kCopyThreads);
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, host_copy_kernel, static_cast<const uint8_t*>(src),
+                         static_cast<uint8_t*>(dst), bytes) != cudaSuccess)
+    return CQ_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+// Whether p is page-locked host memory a kernel can address (registered or
+// allocated by the runtime as pinned).
+static bool device_addressable_host(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();                    // pageable memory may report an error: clear it
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost && a.devicePointer == p;
+}
+
 extern "C" int cq_gemm_host(const uint16_t* x_host, int64_t M, const uint8_t* packed,
                             const float* scales, const uint16_t* ab, int64_t N, int64_t K, int B,
                             int G, int grid_mode, int epilogue, int out_dtype, void* y_host,
@@ -284,14 +339,23 @@ extern "C" int cq_gemm_host(const uint16_t* x_host, int64_t M, const uint8_t* pa
   const size_t x_bytes = static_cast<size_t>(M) * K * 2;
   const int64_t ncol = epilogue == CQ_EPI_SWIGLU ? N / 2 : N;
   const size_t y_bytes = static_cast<size_t>(M) * ncol * (out_dtype == CQ_DTYPE_BF16 ? 2 : 4);
-  if (cudaMemcpyAsync(x_dev, x_host, x_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return CQ_ERR_CUDA;
+  // page-locked buffers on both sides: three chained kernels; otherwise the
+  // copy engine (the driver stages pageable memory itself)
+  const bool kernels = aligned(x_host, 16) && aligned(y_host, 16) &&
+                       device_addressable_host(x_host) && device_addressable_host(y_host);
+  if (kernels) {
+    st = launch_host_copy(x_host, x_dev, static_cast<int64_t>(x_bytes), sms, s);
+  } else {
+    st = cudaMemcpyAsync(x_dev, x_host, x_bytes, cudaMemcpyHostToDevice, s) == cudaSuccess
+             ? CQ_OK : CQ_ERR_CUDA;
+  }
+  if (st != CQ_OK) return st;
   st = gemm_impl(x_dev, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype, y_dev,
                  workspace, ws_bytes, s, kDefaultTimeoutNs, 0);
   if (st != CQ_OK) return st;
-  if (cudaMemcpyAsync(y_host, y_dev, y_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return CQ_ERR_CUDA;
-  return CQ_OK;
+  if (kernels) return launch_host_copy(y_dev, y_host, static_cast<int64_t>(y_bytes), sms, s);
+  return cudaMemcpyAsync(y_host, y_dev, y_bytes, cudaMemcpyDeviceToHost, s) == cudaSuccess
+             ? CQ_OK : CQ_ERR_CUDA;
 }
 
 // Profiling hook (declared in cq_hooks.h): cq_gemm that also writes per-CTA

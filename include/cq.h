@@ -182,10 +182,12 @@ CQ_API int cq_gemm_noalloc(const uint16_t *x, int64_t M, const uint8_t *packed,
  * y_host.  Same arguments, semantics and results as cq_gemm otherwise (the
  * article has no counterpart; this is a calling convenience).
  *   x_host  HOST bfloat16 [M][K]; y_host HOST [M][N] (or [M][N/2] with
- *           SwiGLU) in out_dtype.  Page-locked (pinned) host buffers keep
- *           the copies asynchronous; pageable ones make the driver stage
- *           them synchronously.  Both must stay valid until the stream has
- *           run the call's work.
+ *           SwiGLU) in out_dtype.  When both are page-locked (pinned) and
+ *           16-byte aligned, the copies are small kernels that read and
+ *           write that memory directly, chained to the GEMM by programmatic
+ *           dependent launch; otherwise they go through the copy engine
+ *           (pageable memory is staged by the driver, synchronously).  Both
+ *           must stay valid until the stream has run the call's work.
  *   x_dev   DEVICE staging buffer of M*K*2 bytes; y_dev DEVICE staging
  *           buffer of the output's size; both 16-byte aligned, owned by the
  *           caller (the library allocates nothing).
