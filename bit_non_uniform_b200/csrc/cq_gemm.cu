@@ -265,10 +265,10 @@ extern "C" int cq_gemm(const uint16_t* x, int64_t M, const uint8_t* packed, cons
 }
 
 // ---------------------------------------------------------------------------
-// host-buffer GEMM: copies between page-locked host memory and the device
-// staging buffers as kernels chained to the GEMM by programmatic dependent
-// launch (a copy-engine transfer between two kernels breaks the chain and
-// adds its own start latency on each side)
+// host-buffer GEMM: the copy of x from page-locked host memory as a kernel
+// chained to the GEMM by programmatic dependent launch (a copy-engine
+// transfer before a kernel breaks the chain and adds its own start latency),
+// and the GEMM's stores straight into a page-locked y
 // ---------------------------------------------------------------------------
 constexpr int kCopyThreads = 256;
 
@@ -350,10 +350,11 @@ extern "C" int cq_gemm_host(const uint16_t* x_host, int64_t M, const uint8_t* pa
              ? CQ_OK : CQ_ERR_CUDA;
   }
   if (st != CQ_OK) return st;
-  st = gemm_impl(x_dev, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype, y_dev,
-                 workspace, ws_bytes, s, kDefaultTimeoutNs, 0);
-  if (st != CQ_OK) return st;
-  if (kernels) return launch_host_copy(y_dev, y_host, static_cast<int64_t>(y_bytes), sms, s);
+  // a page-locked y_host takes the GEMM's stores directly (every kernel only
+  // stores to its output); otherwise y_dev is staged and copied back
+  st = gemm_impl(x_dev, M, packed, scales, ab, N, K, B, G, grid_mode, epilogue, out_dtype,
+                 kernels ? y_host : y_dev, workspace, ws_bytes, s, kDefaultTimeoutNs, 0);
+  if (st != CQ_OK || kernels) return st;
   return cudaMemcpyAsync(y_host, y_dev, y_bytes, cudaMemcpyDeviceToHost, s) == cudaSuccess
              ? CQ_OK : CQ_ERR_CUDA;
 }

@@ -183,11 +183,13 @@ CQ_API int cq_gemm_noalloc(const uint16_t *x, int64_t M, const uint8_t *packed,
  * article has no counterpart; this is a calling convenience).
  *   x_host  HOST bfloat16 [M][K]; y_host HOST [M][N] (or [M][N/2] with
  *           SwiGLU) in out_dtype.  When both are page-locked (pinned) and
- *           16-byte aligned, the copies are small kernels that read and
- *           write that memory directly, chained to the GEMM by programmatic
- *           dependent launch; otherwise they go through the copy engine
- *           (pageable memory is staged by the driver, synchronously).  Both
- *           must stay valid until the stream has run the call's work.
+ *           16-byte aligned, x is copied by a small kernel that reads the
+ *           host memory directly, chained to the GEMM by programmatic
+ *           dependent launch, and the GEMM stores its output straight into
+ *           y_host (y_dev is then not used); otherwise both copies go
+ *           through the copy engine (pageable memory is staged by the
+ *           driver, synchronously).  Both must stay valid until the stream
+ *           has run the call's work.
  *   x_dev   DEVICE staging buffer of M*K*2 bytes; y_dev DEVICE staging
  *           buffer of the output's size; both 16-byte aligned, owned by the
  *           caller (the library allocates nothing).
