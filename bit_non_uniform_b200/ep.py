@@ -8,10 +8,11 @@ is the expert-parallel exchange around `cq_moe_grouped_gemm`:
 * the E experts are split over the W ranks of a process group in contiguous
   blocks (rank d owns experts [d E/W, (d+1) E/W));
 * every rank brings its own tokens with their top-k ids and weights;
-* **dispatch**: one all-to-all sends each token row once to every rank that
-  owns at least one of its experts, with its top-k ids made local to that
-  rank (ids of other ranks become -1, which the grouped GEMM drops) and the
-  matching weights (0 elsewhere);
+* **dispatch**: an all-to-all of row counts, then one all-to-all of packed
+  rows sends each token row once to every rank that owns at least one of its
+  experts, together with its top-k ids made local to that rank (ids of other
+  ranks become -1, which the grouped GEMM drops) and the matching weights (0
+  elsewhere): 2H + 8k bytes per row;
 * **compute**: each rank runs the grouped GEMM over the rows it received and
   its own experts, combining the local routes of every row (FP32);
 * **combine**: a second all-to-all returns the partial rows, and each token's
@@ -98,27 +99,29 @@ class MoeExpertParallel:
         dev = tokens.device
         rows, local_ids = self.plan(topk_ids)
         send_n = [int(r.numel()) for r in rows]
-        # dispatch payload: token rows as bytes, then (ids, weight bits) as int32
-        send_x = torch.cat([tokens[r] for r in rows]).view(torch.uint8).reshape(-1, 2 * H)
-        send_m = torch.cat([
-            torch.cat([li, torch.where(li >= 0, topk_w[r], torch.zeros_like(topk_w[r]))
-                       .to(torch.float32).view(torch.int32)], dim=1)
-            for r, li in zip(rows, local_ids)]).reshape(-1, 2 * k)
+        # dispatch payload, one row per (token, destination): the token's 2H
+        # bytes of BF16, then its k local ids and k weight bit patterns
+        # (int32 each), all as bytes
+        row_bytes = 2 * H + 8 * k
+        send = torch.cat([
+            torch.cat([tokens[r].view(torch.uint8).reshape(-1, 2 * H),
+                       li.view(torch.uint8).reshape(-1, 4 * k),
+                       torch.where(li >= 0, topk_w[r], torch.zeros_like(topk_w[r]))
+                       .to(torch.float32).view(torch.uint8).reshape(-1, 4 * k)], dim=1)
+            for r, li in zip(rows, local_ids)]).reshape(-1, row_bytes)
         if self.world == 1:
             recv_n = send_n
-            recv_x, recv_m = send_x, send_m
+            recv = send
         else:
             cnt_out = torch.tensor(send_n, dtype=torch.int64, device=dev)
             cnt_in = torch.empty_like(cnt_out)
             _a2a(cnt_in, cnt_out, [1] * self.world, [1] * self.world, self.group)
             recv_n = [int(v) for v in cnt_in.tolist()]
-            recv_x = torch.empty((sum(recv_n), 2 * H), dtype=torch.uint8, device=dev)
-            recv_m = torch.empty((sum(recv_n), 2 * k), dtype=torch.int32, device=dev)
-            _a2a(recv_x, send_x, recv_n, send_n, self.group)
-            _a2a(recv_m, send_m, recv_n, send_n, self.group)
-        x_in = recv_x.view(torch.bfloat16).reshape(-1, H).contiguous()
-        ids_in = recv_m[:, :k].contiguous()
-        w_in = recv_m[:, k:].contiguous().view(torch.float32)
+            recv = torch.empty((sum(recv_n), row_bytes), dtype=torch.uint8, device=dev)
+            _a2a(recv, send, recv_n, send_n, self.group)
+        x_in = recv[:, :2 * H].contiguous().view(torch.bfloat16)
+        ids_in = recv[:, 2 * H:2 * H + 4 * k].contiguous().view(torch.int32)
+        w_in = recv[:, 2 * H + 4 * k:].contiguous().view(torch.float32)
         part = self.compute(x_in, ids_in, w_in)
         # combine: partials back to the token owners, summed in rank order
         if self.world == 1:
