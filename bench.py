@@ -414,11 +414,15 @@ def time_cold(cq, name, device):
 
 
 MOE_WORKLOADS = {
-    # name: (description, T, routing, widths)
+    # name: (description, T, routing, widths, experts)
     "moe_decode": ("Kimi-K3 MoE layer, 896 experts W2/W3/W4 (P=.6/.3/.1) G512, 64 tokens, "
-                   "uniform top-16", 64, "uniform", "mixed"),
+                   "uniform top-16", 64, "uniform", "mixed", 896),
     "moe_prefill": ("Kimi-K3 MoE layer, 896 experts W4 G512, 8192 tokens, Zipf(1.1) top-16",
-                    8192, "zipf", "w4"),
+                    8192, "zipf", "w4", 896),
+    # the decode layer's kernels on 64 of its experts (1.3 GB of weights: a size an ncu
+    # capture with every counter can replay); not a bench line
+    "moe_decode_64e": ("Kimi-K3 MoE layer shapes, 64 experts W2/W3/W4 (P=.6/.3/.1) G512, "
+                       "16 tokens, uniform top-16", 16, "uniform", "mixed", 64),
 }
 
 
@@ -426,8 +430,8 @@ def time_moe(cq, name, steps, device):
     """Device-timed steps of one MoE layer (routing, gather, gate/up, down,
     combine), captured in a CUDA graph; inputs and weights resident."""
     import synthetic
-    desc, T, routing, widths = MOE_WORKLOADS[name]
-    H, I, E, k, G = 7168, 3072, 896, 16, 512
+    desc, T, routing, widths, E = MOE_WORKLOADS[name]
+    H, I, k, G = 7168, 3072, 16, 512
     Bs = synthetic.expert_bits(4, E) if widths == "mixed" else torch.full((E,), 4)
     experts = []
     for e in range(E):
@@ -696,6 +700,8 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-moe", action="store_true")
+    ap.add_argument("--moe-only", choices=sorted(MOE_WORKLOADS),
+                    help="time one MoE layer and print its line only (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -709,6 +715,14 @@ def main():
     world, rank, local = dist_setup(args)
     device = torch.device("cuda", torch.cuda.current_device())
     hbm, tf_burst, tf_sust, peak_src = load_peaks()
+    if args.moe_only:
+        r = time_moe(cq, args.moe_only, max(args.steps, 1), device)
+        if rank == 0:
+            print(json.dumps({"workload": r["desc"], "ms_per_step": round(r["ms"], 4),
+                              "active_weight_bytes": r["wbytes"],
+                              "packed_gbs": round(r["gbs"], 1), "tflops": round(r["tflops"], 2),
+                              "frac_hbm": round(r["gbs"] / hbm, 4)}))
+        return 0
 
     main_res = time_gemm(cq, args.workload, args.steps, args.warmup, world, device,
                          sample_clocks=True, repeats=20)
